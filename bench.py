@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Benchmark of the VSA forward path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the whole path over one batch: tile q, k, v into
+cubes; coarse stage (pool, coarse attention, top-k); fine block-sparse
+attention; gated combine; untile.  Inputs are drawn once on the host from the
+seeded synthetic recipe and are resident in HBM before the timed region; each
+input tensor (774 MB at the default workload) is larger than the 126 MB L2,
+so no flush is needed between steps.
+
+Metric: effective TFLOP/s of the whole call, counting only the FLOPs the
+chosen sparsity needs: 4*d*sum_i n_i*sum_{j in sel(i)} n_j for the fine stage
+(valid tokens of the actual selection) plus 4*d*C^2 per head for the coarse
+attention.  ms/call is ``ms_per_step``.
+
+Prints ONE JSON line on rank 0.  With ``--impl reference`` the same metric is
+measured for the CPU oracle (float64 NumPy) on a bounded sample of the
+workload on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from video_dit_block_vsa_b200 import workloads as wl  # noqa: E402
+
+DEFAULT_WORKLOAD = "wan14b_720p_21x45x80_k180"
+METRIC = "block-sparse attention ms/call & effective TFLOP/s (% bf16 peak), 1 B200"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sustained=p["bf16_tflops_sustained"],
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def cube_counts(grid):
+    """Valid tokens per cube for a 4x4x4 tiling (bench accounting only)."""
+    T, Y, X = grid
+    ct = np.minimum(4, T - 4 * np.arange(-(-T // 4)))
+    cy = np.minimum(4, Y - 4 * np.arange(-(-Y // 4)))
+    cx = np.minimum(4, X - 4 * np.arange(-(-X // 4)))
+    return (ct[:, None, None] * cy[None, :, None] * cx[None, None, :]).reshape(-1).astype(np.int64)
+
+
+def flop_counts(w, counts, sel):
+    """(fine effective FLOPs, fine issued FLOPs, coarse FLOPs) of one call."""
+    d, C = w.head_dim, counts.shape[0]
+    nsel = counts[sel]                         # [B, H, C, k]
+    fine_eff = 4.0 * d * float(np.sum(counts[None, None, :] * nsel.sum(axis=-1)))
+    fine_issued = 4.0 * d * w.batch * w.heads * C * w.topk * 64 * 64
+    coarse = 4.0 * d * w.batch * w.heads * C * C
+    return fine_eff, fine_issued, coarse
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ oracle (CPU)
+
+def oracle_sample(w, x, time_budget_s, cubes_cap=None):
+    """Runs the oracle on head 0 of batch 0: the whole coarse stage, then the
+    fine stage for query cubes in order until the time budget or the cap.
+    Returns (seconds, effective FLOPs processed, description)."""
+    from oracle import vsa_oracle as vo
+    t0 = time.perf_counter()
+    one = lambda n: vo.bf16_bits_to_f64(x[n][0:1, 0:1])
+    q_t, counts = vo.tile_permute(one("q"), w.grid)
+    k_t, _ = vo.tile_permute(one("k"), w.grid)
+    v_t, _ = vo.tile_permute(one("v"), w.grid)
+    S, O_c = vo.coarse_attention(vo.pool(q_t, counts), vo.pool(k_t, counts), vo.pool(v_t, counts))
+    sel = vo.topk_select(S, w.topk)
+    C, d = counts.shape[0], w.head_dim
+    flops = 4.0 * d * C * C
+    done = 0
+    while done < C and (cubes_cap is None or done < cubes_cap):
+        vo.block_sparse_attention(q_t, k_t, v_t, counts, sel, query_cubes=[done])
+        flops += 4.0 * d * counts[done] * counts[sel[0, 0, done]].sum()
+        done += 1
+        if time.perf_counter() - t0 > time_budget_s:
+            break
+    dt = time.perf_counter() - t0
+    desc = (f"head 0 of {w.batch * w.heads}: tile/pool/coarse/top-k over all {C} cubes, "
+            f"fine stage for query cubes 0..{done - 1} ({done} of {C})")
+    return dt, flops, desc
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:  # pragma: no cover
+        return os.cpu_count()
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    x = wl.make_inputs(w, heads=1)
+    per_step_budget = 8.0
+    for _ in range(args.warmup):
+        oracle_sample(w, x, per_step_budget, cubes_cap=4)
+    tot_t = tot_f = 0.0
+    desc = ""
+    for _ in range(args.steps):
+        dt, fl, desc = oracle_sample(w, x, per_step_budget)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": desc + f"; input draw limited to head 0; {args.steps} steps"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w):
+    C = w.cubes
+    return {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
+            "grid": list(w.grid), "tokens": w.tokens, "cubes": C, "topk": w.topk,
+            "sparsity": round(1.0 - w.topk / C, 4), "gated": w.gated,
+            "l2": "inputs larger than L2 (no flush)"}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_gpu(args, w):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+
+    from video_dit_block_vsa_b200 import vsa
+
+    peaks = load_peaks()
+    x = wl.make_inputs(w)
+    shape = vsa.make_shape(w.batch, w.heads, w.head_dim, w.grid)
+    dev = torch.device("cuda", local)
+    to_dev = lambda b: torch.from_numpy(b.view(np.int16)).to(dev).view(torch.bfloat16)
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    g_f = torch.from_numpy(x["g_f"]).to(dev) if w.gated else None
+    g_c = torch.from_numpy(x["g_c"]).to(dev) if w.gated else None
+    out = torch.empty_like(q)
+    bufs = vsa.VsaBuffers(shape, w.topk, device=dev, want_coarse=w.gated)
+    stream = torch.cuda.current_stream()
+
+    stages = ["tile_permute", "coarse_select", "block_sparse_fwd", "combine", "untile"]
+
+    def step(ev=None):
+        def mark(i):
+            if ev is not None:
+                ev[i].record(stream)
+        mark(0)
+        vsa.vsa_tile_permute(shape, q, bufs.q_t, bufs.counts)
+        vsa.vsa_tile_permute(shape, k, bufs.k_t)
+        vsa.vsa_tile_permute(shape, v, bufs.v_t)
+        mark(1)
+        vsa.vsa_coarse_select(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, w.topk, bufs.sel,
+                              bufs.workspace, o_coarse=bufs.o_c)
+        mark(2)
+        vsa.vsa_block_sparse_fwd(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, bufs.sel,
+                                 w.topk, bufs.o_f)
+        mark(3)
+        vsa.vsa_combine(shape, bufs.o_f, bufs.o_f, bufs.o_c, g_f, g_c)  # in place
+        mark(4)
+        vsa.vsa_untile(shape, bufs.o_f, out)
+        mark(5)
+
+    launches_per_step = 3 + 2 + 1 + (1 if w.gated else 0) + 1
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    status = vsa.vsa_get_status()
+    if status != 0:
+        raise RuntimeError(f"device status after warm-up: {vsa.vsa_strerror(status)}")
+    counts = cube_counts(w.grid)
+    fine_eff, fine_issued, coarse_fl = flop_counts(w, counts, bufs.sel.cpu().numpy().astype(np.int64))
+    step_flops = fine_eff + coarse_fl
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    status = vsa.vsa_get_status()
+    if status != 0:
+        raise RuntimeError(f"device status after timed steps: {vsa.vsa_strerror(status)}")
+    stage_ms = {name: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps))
+                for i, name in enumerate(stages)}
+    ms_per_step = elapsed_ms / args.steps
+    value = world * step_flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+
+    # ---- end to end through host buffers (pinned), copies inside the timed region
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hgf = g_f.cpu().pin_memory() if w.gated else None
+    hgc = g_c.cpu().pin_memory() if w.gated else None
+    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        if w.gated:
+            g_f.copy_(hgf, non_blocking=True)
+            g_c.copy_(hgc, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    if w.gated:
+        h2d += hgf.numel() * 4 + hgc.numel() * 4
+    d2h = hout.numel() * hout.element_size()
+
+    # ---- roofline of the dominant kernel (fine block-sparse attention)
+    fine_ms = stage_ms["block_sparse_fwd"]
+    achieved = fine_eff / (fine_ms * 1e-3) / 1e12
+    traffic_path = os.path.join(ROOT, "profiles", "fine_traffic.json")
+    traffic = None
+    try:
+        with open(traffic_path) as f:
+            tj = json.load(f)
+        if tj.get("workload") == w.name and tj.get("kernel_rev") == KERNEL_REV:
+            traffic = tj.get("bytes_per_launch")
+    except (OSError, ValueError):
+        pass
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_sustained"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"], "traffic": traffic,
+                "kernel": "vsa_block_sparse_fwd", "peak_kind": f"bf16 sustained ({peaks['source']})",
+                "peak_burst": peaks["bf16"], "frac_of_burst": achieved / peaks["bf16"],
+                "issued_tflops": fine_issued / (fine_ms * 1e-3) / 1e12}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, fl, desc = oracle_sample(w, x, args.cpu_seconds)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+               "kind": "oracle", "sample": desc + f", {dt:.1f} s"}
+
+    if rank == 0:
+        hbm_bytes = {
+            "tile_permute": 3 * w.batch * w.heads * (w.tokens + 64 * w.cubes) * w.head_dim * 2,
+            "untile": w.batch * w.heads * (w.tokens + 64 * w.cubes) * w.head_dim * 2,
+        }
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) + per-cube mean N(0,0.5^2), bf16)",
+            "config": config_dict(w),
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * step_flops * args.steps / (e2e_ms * 1e-3) / 1e12,
+                    "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms / args.steps},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+            "stages_ms": stage_ms,
+            "stages_gbs": {k: v / (stage_ms[k] * 1e-3) / 1e9 for k, v in hbm_bytes.items()},
+            "flops": {"fine_effective": fine_eff, "fine_issued": fine_issued, "coarse": coarse_fl},
+            "kernel_rev": KERNEL_REV,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+# Revision tag of the fine kernel; ncu traffic figures are only reported for
+# the revision they were captured on.
+KERNEL_REV = "fine-v0"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = wl.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,168 @@
+/*
+ * vsa.h -- C ABI of the B200 (sm_100a) video sparse attention (VSA) forward path.
+ *
+ * VSA is the trainable, dynamic block-sparse attention of FastWan ("单块 H200
+ * ... 5 秒即生一个 5 秒视频", section "一张卡，秒生视频"; restated in
+ * "超越Sora：FastWan如何以“稀疏蒸馏”重塑实时AI视频生成范式", section
+ * "技术原理与创新点解析").  A coarse stage looks at the whole sequence at
+ * block granularity and picks, for every query block, the key blocks that
+ * matter; a fine block-sparse kernel then runs exact attention over those
+ * 64x64 blocks only.  The pages name the stages but print no formula; the
+ * readings taken here are stated with each call.
+ *
+ * Terms
+ *   B       batch, H heads, d head dim (64 or 128)
+ *   grid    latent token grid T x Hg x Wg; N = T*Hg*Wg tokens in row-major
+ *           (t, y, x) order, token n = (t*Hg + y)*Wg + x
+ *   cube    4x4x4 block of the grid = 64 token slots.  Cube c = (ct*Cy+cy)*Cx+cx
+ *           with Ct = ceil(T/4), Cy = ceil(Hg/4), Cx = ceil(Wg/4), C = Ct*Cy*Cx.
+ *           Edge cubes of a grid whose sides are not multiples of 4 are
+ *           partial: they hold n_c < 64 tokens.
+ *   tiled   [B, H, 64*C, d] layout: cube c owns rows 64c .. 64c+63; its n_c
+ *           tokens fill the first n_c rows in row-major local (t, y, x)
+ *           order; the remaining rows are zero padding.
+ *   k       number of key cubes each query cube attends to (1 <= k <= C).
+ *
+ * Conventions (every call)
+ *   - Tensor pointers are DEVICE pointers owned by the caller, contiguous
+ *     row-major, 16-byte aligned.  bf16 tensors are IEEE bfloat16 bit
+ *     patterns.  The library allocates no device memory; scratch comes from
+ *     the caller's workspace (vsa_coarse_select).
+ *   - Every call is asynchronous on `stream`.  A call returns VSA_OK after a
+ *     successful launch; argument errors are reported before any launch and
+ *     nothing is written.
+ *   - Device-side conditions (a bounded wait that ran out, an inconsistent
+ *     cube_count / sel_idx entry) are recorded in a per-device status word
+ *     read and cleared by vsa_get_status().  Kernels never trap.
+ *   - Calls on one device from several host threads are safe; calls that
+ *     overlap on the GPU and write the same output race, as any CUDA kernel.
+ */
+#ifndef VSA_H_
+#define VSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum vsa_status_code {
+  VSA_OK = 0,
+  VSA_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, bad size, k not in [1, C] */
+  VSA_ERR_UNSUPPORTED = 2,  /* cube not 4x4x4, d not in {64, 128}, device not sm_100 */
+  VSA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  VSA_ERR_TIMEOUT = 4,      /* device: a bounded wait ran out (status word) */
+  VSA_ERR_BAD_INDEX = 5     /* device: cube_count or sel_idx entry inconsistent (status word) */
+};
+
+typedef struct vsa_shape {
+  int batch;                       /* B >= 1 */
+  int heads;                       /* H >= 1 */
+  int head_dim;                    /* d: 64 or 128 */
+  int grid_t, grid_h, grid_w;      /* latent token grid, each >= 1 */
+  int cube_t, cube_h, cube_w;      /* must be 4, 4, 4 */
+} vsa_shape;
+
+/* Host-only helper: C = ceil(T/4)*ceil(Hg/4)*ceil(Wg/4).  No GPU work. */
+int vsa_num_cubes(const vsa_shape* shape, int* num_cubes);
+
+/* Host-only helper: k from a top-k ratio r of the C cubes,
+ * k = max(1, floor(r*C + 0.5)).  A ratio of 0.1 is the 90 % attention
+ * sparsity of the TurboDiffusion review (section "評估 / 設置"); 0.125 is the
+ * 87.5 % sparsity of the FastWan scaling experiment.  r must be in (0, 1]. */
+int vsa_topk_from_ratio(int num_cubes, float ratio, int* topk);
+
+/* Bytes of device workspace vsa_coarse_select needs for this shape and k
+ * (pooled q, k, v in float32: 3*B*H*C*d*4 bytes, rounded up to 256). */
+size_t vsa_workspace_bytes(const vsa_shape* shape, int topk);
+
+/* Token -> cube permutation (the 4x4x4 tiling the coarse and fine stages
+ * work on; 64-token blocks are the 64x64 blocks of the fine kernel).
+ *   x          bf16 [B, H, N, d], token order           (read)
+ *   x_tiled    bf16 [B, H, 64*C, d], tiled; pad rows 0  (written)
+ *   cube_count int32 [C] valid tokens per cube, or NULL (written)
+ * One call per tensor (q, k, v). */
+int vsa_tile_permute(const vsa_shape* shape, const void* x, void* x_tiled,
+                     int32_t* cube_count, cudaStream_t stream);
+
+/* Coarse stage (FastWan article, section "一张卡，秒生视频", Fig. 5
+ * paragraph: the block-sparse attention the coarse stage produces is highly
+ * dynamic).  Reading taken: each cube is mean-pooled over its n_c valid
+ * tokens (qbar, kbar, vbar); coarse attention over the C pooled vectors with
+ * scale 1/sqrt(d) gives the coarse output O_c = softmax(qbar kbar^T/sqrt(d)) vbar;
+ * for each query cube the k key cubes with the largest coarse logits are
+ * selected, ties to the lower index, listed in ascending index order.
+ * Logits are computed in float32.
+ *   q_tiled, k_tiled, v_tiled  bf16 [B, H, 64*C, d] from vsa_tile_permute
+ *   cube_count   int32 [C] as written by vsa_tile_permute for this shape
+ *                (checked against the grid; a mismatch is recorded as
+ *                VSA_ERR_BAD_INDEX and the grid's count is used)
+ *   topk         k, 1 <= k <= C
+ *   o_coarse     float32 [B, H, C, d] coarse output, or NULL
+ *   sel_idx      int32 [B, H, C, k] selected key cubes (written)
+ *   coarse_logits float32 [B, H, C, C] scaled logits, or NULL (diagnostics)
+ *   workspace    device scratch of at least vsa_workspace_bytes(shape, k)
+ *                bytes, 256-byte aligned; contents on entry are ignored */
+int vsa_coarse_select(const vsa_shape* shape, const void* q_tiled, const void* k_tiled,
+                      const void* v_tiled, const int32_t* cube_count, int topk,
+                      float* o_coarse, int32_t* sel_idx, float* coarse_logits,
+                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Fine stage: block-sparse attention over the selected 64x64 blocks (FastWan
+ * article, section "一张卡，秒生视频": the fine block-sparse kernel, 64x64
+ * block mask).  For every valid query token r of cube i:
+ *   O_f[r] = softmax_t(q_r . k_t / sqrt(d)) v_t  over the valid tokens t of
+ * the cubes in sel_idx[b, h, i, :].  Pad key slots are masked out; pad query
+ * rows are written as 0.  bf16 in, float32 accumulation, bf16 out.
+ *   q_tiled, k_tiled, v_tiled  bf16 [B, H, 64*C, d]
+ *   cube_count   int32 [C] (checked as in vsa_coarse_select)
+ *   sel_idx      int32 [B, H, C, k], each row strictly ascending in [0, C)
+ *                (an entry out of range or out of order is recorded as
+ *                VSA_ERR_BAD_INDEX; out-of-range entries are clamped)
+ *   o_fine_tiled bf16 [B, H, 64*C, d] (written)
+ *   lse          float32 [B, H, 64*C] natural-log log-sum-exp of each valid
+ *                row's scaled scores (-inf for pad rows), or NULL */
+int vsa_block_sparse_fwd(const vsa_shape* shape, const void* q_tiled, const void* k_tiled,
+                         const void* v_tiled, const int32_t* cube_count,
+                         const int32_t* sel_idx, int topk, void* o_fine_tiled,
+                         float* lse, cudaStream_t stream);
+
+/* Optional per-token gated sum of the fine and coarse outputs, in tiled order:
+ *   out[r] = g_fine[n] * O_f[r] + g_coarse[n] * O_c[cube of r]
+ * where n is the token held by tiled row r.  With g_fine == g_coarse == NULL,
+ * out = O_f (a copy).  Either both gates are given or neither.
+ *   o_fine_tiled bf16 [B, H, 64*C, d]
+ *   o_coarse     float32 [B, H, C, d] (may be NULL when the gates are NULL)
+ *   g_fine, g_coarse float32 [B, H, N] in TOKEN order, or both NULL
+ *   out_tiled    bf16 [B, H, 64*C, d]; pad rows 0 (may alias o_fine_tiled) */
+int vsa_combine(const vsa_shape* shape, const void* o_fine_tiled, const float* o_coarse,
+                const float* g_fine, const float* g_coarse, void* out_tiled,
+                cudaStream_t stream);
+
+/* Inverse of vsa_tile_permute: bf16 [B, H, 64*C, d] -> bf16 [B, H, N, d];
+ * pad rows are dropped. */
+int vsa_untile(const vsa_shape* shape, const void* x_tiled, void* x, cudaStream_t stream);
+
+/* Synchronises `stream`, then returns and clears the status word of the
+ * current device: VSA_OK, VSA_ERR_TIMEOUT or VSA_ERR_BAD_INDEX recorded by a
+ * kernel since the last call, or VSA_ERR_CUDA if the synchronisation failed. */
+int vsa_get_status(cudaStream_t stream);
+
+/* Diagnostic: launches one kernel that waits on a barrier nothing arrives at,
+ * for at most timeout_ns nanoseconds (1e3 .. 1e9), with the same bounded wait
+ * the fine kernel uses; it then records VSA_ERR_TIMEOUT in the status word and
+ * returns, leaving the context usable.  Used by the tests to exercise the
+ * timeout path without faulting the GPU. */
+int vsa_debug_wait_timeout(uint64_t timeout_ns, cudaStream_t stream);
+
+/* Static text for a status code. */
+const char* vsa_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H_ */

@@ -1,0 +1,97 @@
+"""libvsa on a machine without a GPU: the library builds, loads, exports every
+symbol include/vsa.h declares, and its host-only helpers and argument checks
+work (no call here launches GPU work)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "vsa.h")
+
+
+@pytest.fixture(scope="module")
+def vsa():
+    from video_dit_block_vsa_b200 import build
+    build.build()
+    from video_dit_block_vsa_b200 import vsa as mod
+    return mod
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(vsa_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for n in ("vsa_tile_permute", "vsa_coarse_select", "vsa_block_sparse_fwd", "vsa_combine",
+              "vsa_untile"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(vsa):
+    lib = ctypes.CDLL(vsa._LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    assert set(declared_functions()) == set(vsa.EXPORTED)
+
+
+def test_num_cubes_and_ratio(vsa):
+    s = vsa.make_shape(1, 40, 128, (21, 45, 80))
+    assert vsa.vsa_num_cubes(s) == 1440
+    assert vsa.vsa_num_cubes(vsa.make_shape(1, 12, 128, (21, 30, 52))) == 624
+    assert vsa.vsa_topk_from_ratio(624, 0.1) == 62
+    assert vsa.vsa_topk_from_ratio(1440, 0.125) == 180
+    assert vsa.vsa_topk_from_ratio(1440, 0.03) == 43
+    assert vsa.vsa_topk_from_ratio(1440, 1.0) == 1440
+    with pytest.raises(vsa.VsaError):
+        vsa.vsa_topk_from_ratio(1440, 0.0)
+    with pytest.raises(vsa.VsaError):
+        vsa.vsa_topk_from_ratio(0, 0.5)
+
+
+def test_workspace_bytes(vsa):
+    s = vsa.make_shape(1, 40, 128, (21, 45, 80))
+    assert vsa.vsa_workspace_bytes(s, 180) == 3 * 40 * 1440 * 128 * 4
+    assert vsa.vsa_workspace_bytes(s, 0) == 0
+    assert vsa.vsa_workspace_bytes(s, 1441) == 0
+
+
+def test_unsupported_shapes_rejected_before_launch(vsa):
+    lib = vsa._lib
+    c = ctypes.c_int()
+    bad_cube = vsa.VsaShape(1, 1, 128, 8, 8, 8, 2, 4, 4)
+    assert lib.vsa_num_cubes(ctypes.byref(bad_cube), ctypes.byref(c)) == vsa.VSA_ERR_UNSUPPORTED
+    bad_d = vsa.make_shape(1, 1, 96, (8, 8, 8))
+    assert lib.vsa_num_cubes(ctypes.byref(bad_d), ctypes.byref(c)) == vsa.VSA_ERR_UNSUPPORTED
+    bad_b = vsa.make_shape(0, 1, 128, (8, 8, 8))
+    assert lib.vsa_num_cubes(ctypes.byref(bad_b), ctypes.byref(c)) == vsa.VSA_ERR_INVALID_ARG
+    assert lib.vsa_num_cubes(None, ctypes.byref(c)) == vsa.VSA_ERR_INVALID_ARG
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch(vsa):
+    lib = vsa._lib
+    s = vsa.make_shape(1, 2, 64, (4, 8, 8))
+    p = ctypes.c_void_p(0x1000)
+    odd = ctypes.c_void_p(0x1008)
+    assert lib.vsa_tile_permute(ctypes.byref(s), None, p, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert lib.vsa_tile_permute(ctypes.byref(s), odd, p, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert lib.vsa_untile(ctypes.byref(s), p, None, None) == vsa.VSA_ERR_INVALID_ARG
+    # k outside [1, C]
+    assert lib.vsa_block_sparse_fwd(ctypes.byref(s), p, p, p, p, p, 0, p, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert lib.vsa_block_sparse_fwd(ctypes.byref(s), p, p, p, p, p, 5, p, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert lib.vsa_coarse_select(ctypes.byref(s), p, p, p, p, 5, None, p, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
+    # workspace too small
+    assert lib.vsa_coarse_select(ctypes.byref(s), p, p, p, p, 2, None, p, None, p, 16, None) == vsa.VSA_ERR_INVALID_ARG
+    # one gate without the other
+    assert lib.vsa_combine(ctypes.byref(s), p, p, p, None, p, None) == vsa.VSA_ERR_INVALID_ARG
+    assert lib.vsa_debug_wait_timeout(10, None) == vsa.VSA_ERR_INVALID_ARG
+
+
+def test_strerror(vsa):
+    assert vsa.vsa_strerror(0) == "ok"
+    assert "timed out" in vsa.vsa_strerror(vsa.VSA_ERR_TIMEOUT)
+    assert vsa.vsa_strerror(99) == "unknown status"

@@ -1,0 +1,291 @@
+// extern "C" entry points of libvsa (declared in include/vsa.h): argument
+// validation, per-device setup (architecture check, status word address),
+// TMA tensor maps, and the kernel launches of the VSA forward path.
+#include <cuda.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace vsa {
+
+// Launchers (permute.cu, coarse.cu, fine.cu).
+cudaError_t launch_tile_permute(const Geom&, const void*, void*, int32_t*, int, cudaStream_t);
+cudaError_t launch_untile(const Geom&, const void*, void*, int, cudaStream_t);
+cudaError_t launch_combine(const Geom&, const void*, const float*, const float*, const float*,
+                           void*, int, cudaStream_t);
+cudaError_t launch_coarse_select(const Geom&, const void*, const void*, const void*,
+                                 const int32_t*, int, float*, int32_t*, float*, float*, int*,
+                                 cudaStream_t);
+cudaError_t launch_block_sparse_fwd(const Geom&, const CUtensorMap&, const CUtensorMap&,
+                                    const CUtensorMap&, const int32_t*, const int32_t*, int,
+                                    void*, float*, int*, cudaStream_t);
+cudaError_t launch_debug_wait(uint64_t, int*, cudaStream_t);
+
+// Device-side status word, one per device that loads the library.
+__device__ int g_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  int supported = 0;
+  int sms = 0;
+  int* status = nullptr;  // device address of g_status
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Per-device setup on first use: architecture check and the status word's
+// device address (a host-side symbol is not a device pointer).
+int device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return VSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return VSA_ERR_CUDA;
+    st.supported = (major == 10 && minor == 0);
+    st.sms = sms;
+    if (st.supported) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return VSA_ERR_CUDA;
+      st.status = static_cast<int*>(p);
+    }
+    st.ready = true;
+  }
+  if (!st.supported) return VSA_ERR_UNSUPPORTED;
+  *out = &st;
+  return VSA_OK;
+}
+
+int get_encoder() {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_encode) return VSA_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return VSA_ERR_CUDA;
+  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  return VSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validates the shape and fills the geometry.  The tiled row count of all
+// heads must fit a 32-bit TMA coordinate.
+int make_geom(const vsa_shape* s, Geom* g) {
+  if (s == nullptr) return VSA_ERR_INVALID_ARG;
+  if (s->cube_t != 4 || s->cube_h != 4 || s->cube_w != 4) return VSA_ERR_UNSUPPORTED;
+  if (s->head_dim != 64 && s->head_dim != 128) return VSA_ERR_UNSUPPORTED;
+  if (s->batch < 1 || s->heads < 1 || s->grid_t < 1 || s->grid_h < 1 || s->grid_w < 1)
+    return VSA_ERR_INVALID_ARG;
+  g->B = s->batch;
+  g->H = s->heads;
+  g->d = s->head_dim;
+  g->T = s->grid_t;
+  g->Y = s->grid_h;
+  g->X = s->grid_w;
+  g->Ct = (g->T + 3) / 4;
+  g->Cy = (g->Y + 3) / 4;
+  g->Cx = (g->X + 3) / 4;
+  const long long C = static_cast<long long>(g->Ct) * g->Cy * g->Cx;
+  if (C > kMaxCubes) return VSA_ERR_UNSUPPORTED;
+  g->C = static_cast<int>(C);
+  g->N = static_cast<long long>(g->T) * g->Y * g->X;
+  g->rows = C * kSlots;
+  const long long all_rows = static_cast<long long>(g->B) * g->H * g->rows;
+  if (all_rows >= (1ll << 31) || static_cast<long long>(g->B) * g->H >= 65536)
+    return VSA_ERR_UNSUPPORTED;
+  return VSA_OK;
+}
+
+int tiled_map(const Geom& g, const void* ptr, CUtensorMap* m) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(g.d),
+                              static_cast<cuuint64_t>(g.B) * g.H * g.rows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(g.d) * 2};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA; }
+
+}  // namespace
+}  // namespace vsa
+
+using namespace vsa;
+
+extern "C" {
+
+int vsa_num_cubes(const vsa_shape* shape, int* num_cubes) {
+  Geom g;
+  if (num_cubes == nullptr) return VSA_ERR_INVALID_ARG;
+  const int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  *num_cubes = g.C;
+  return VSA_OK;
+}
+
+int vsa_topk_from_ratio(int num_cubes, float ratio, int* topk) {
+  if (topk == nullptr || num_cubes < 1 || !(ratio > 0.0f) || ratio > 1.0f)
+    return VSA_ERR_INVALID_ARG;
+  long long k = static_cast<long long>(std::floor(static_cast<double>(ratio) * num_cubes + 0.5));
+  if (k < 1) k = 1;
+  if (k > num_cubes) k = num_cubes;
+  *topk = static_cast<int>(k);
+  return VSA_OK;
+}
+
+size_t vsa_workspace_bytes(const vsa_shape* shape, int topk) {
+  Geom g;
+  if (make_geom(shape, &g) != VSA_OK || topk < 1 || topk > g.C) return 0;
+  const size_t bytes = 3ull * g.B * g.H * g.C * g.d * sizeof(float);
+  return (bytes + 255) & ~static_cast<size_t>(255);
+}
+
+int vsa_tile_permute(const vsa_shape* shape, const void* x, void* x_tiled, int32_t* cube_count,
+                     cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (!x || !x_tiled || !aligned16(x) || !aligned16(x_tiled) ||
+      (cube_count && (reinterpret_cast<uintptr_t>(cube_count) & 3u)))
+    return VSA_ERR_INVALID_ARG;
+  DeviceState* st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  return cuda_rc(launch_tile_permute(g, x, x_tiled, cube_count, st->sms, stream));
+}
+
+int vsa_untile(const vsa_shape* shape, const void* x_tiled, void* x, cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (!x || !x_tiled || !aligned16(x) || !aligned16(x_tiled)) return VSA_ERR_INVALID_ARG;
+  DeviceState* st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  return cuda_rc(launch_untile(g, x_tiled, x, st->sms, stream));
+}
+
+int vsa_combine(const vsa_shape* shape, const void* o_fine_tiled, const float* o_coarse,
+                const float* g_fine, const float* g_coarse, void* out_tiled, cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (!o_fine_tiled || !out_tiled || !aligned16(o_fine_tiled) || !aligned16(out_tiled))
+    return VSA_ERR_INVALID_ARG;
+  if ((g_fine == nullptr) != (g_coarse == nullptr)) return VSA_ERR_INVALID_ARG;
+  if (g_fine && (!o_coarse || !aligned16(o_coarse) ||
+                 (reinterpret_cast<uintptr_t>(g_fine) & 3u) ||
+                 (reinterpret_cast<uintptr_t>(g_coarse) & 3u)))
+    return VSA_ERR_INVALID_ARG;
+  DeviceState* st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  return cuda_rc(launch_combine(g, o_fine_tiled, o_coarse, g_fine, g_coarse, out_tiled, st->sms,
+                                stream));
+}
+
+int vsa_coarse_select(const vsa_shape* shape, const void* q_tiled, const void* k_tiled,
+                      const void* v_tiled, const int32_t* cube_count, int topk, float* o_coarse,
+                      int32_t* sel_idx, float* coarse_logits, void* workspace,
+                      size_t workspace_bytes, cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (topk < 1 || topk > g.C) return VSA_ERR_INVALID_ARG;
+  if (!q_tiled || !k_tiled || !v_tiled || !cube_count || !sel_idx || !workspace)
+    return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q_tiled) || !aligned16(k_tiled) || !aligned16(v_tiled) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (reinterpret_cast<uintptr_t>(cube_count) & 3u) ||
+      (reinterpret_cast<uintptr_t>(sel_idx) & 3u) || (o_coarse && !aligned16(o_coarse)) ||
+      (coarse_logits && (reinterpret_cast<uintptr_t>(coarse_logits) & 3u)))
+    return VSA_ERR_INVALID_ARG;
+  if (workspace_bytes < vsa_workspace_bytes(shape, topk)) return VSA_ERR_INVALID_ARG;
+  DeviceState* st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  return cuda_rc(launch_coarse_select(g, q_tiled, k_tiled, v_tiled, cube_count, topk, o_coarse,
+                                      sel_idx, coarse_logits, static_cast<float*>(workspace),
+                                      st->status, stream));
+}
+
+int vsa_block_sparse_fwd(const vsa_shape* shape, const void* q_tiled, const void* k_tiled,
+                         const void* v_tiled, const int32_t* cube_count, const int32_t* sel_idx,
+                         int topk, void* o_fine_tiled, float* lse, cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (topk < 1 || topk > g.C) return VSA_ERR_INVALID_ARG;
+  if (!q_tiled || !k_tiled || !v_tiled || !cube_count || !sel_idx || !o_fine_tiled)
+    return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q_tiled) || !aligned16(k_tiled) || !aligned16(v_tiled) ||
+      !aligned16(o_fine_tiled) || (reinterpret_cast<uintptr_t>(cube_count) & 3u) ||
+      (reinterpret_cast<uintptr_t>(sel_idx) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return VSA_ERR_INVALID_ARG;
+  DeviceState* st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  if ((rc = get_encoder()) != VSA_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  if (tiled_map(g, q_tiled, &tq) != VSA_OK || tiled_map(g, k_tiled, &tk) != VSA_OK ||
+      tiled_map(g, v_tiled, &tv) != VSA_OK)
+    return VSA_ERR_CUDA;
+  return cuda_rc(launch_block_sparse_fwd(g, tq, tk, tv, cube_count, sel_idx, topk, o_fine_tiled,
+                                         lse, st->status, stream));
+}
+
+int vsa_get_status(cudaStream_t stream) {
+  DeviceState* st;
+  int rc = device_state(&st);
+  if (rc != VSA_OK) return rc;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return VSA_ERR_CUDA;
+  int value = 0;
+  const int zero = 0;
+  if (cudaMemcpy(&value, st->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(st->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return VSA_ERR_CUDA;
+  return value;
+}
+
+int vsa_debug_wait_timeout(uint64_t timeout_ns, cudaStream_t stream) {
+  if (timeout_ns < 1000ull || timeout_ns > 1000000000ull) return VSA_ERR_INVALID_ARG;
+  DeviceState* st;
+  const int rc = device_state(&st);
+  if (rc != VSA_OK) return rc;
+  return cuda_rc(launch_debug_wait(timeout_ns, st->status, stream));
+}
+
+const char* vsa_strerror(int code) {
+  switch (code) {
+    case VSA_OK: return "ok";
+    case VSA_ERR_INVALID_ARG: return "invalid argument";
+    case VSA_ERR_UNSUPPORTED: return "unsupported shape or device";
+    case VSA_ERR_CUDA: return "CUDA runtime error";
+    case VSA_ERR_TIMEOUT: return "device wait timed out";
+    case VSA_ERR_BAD_INDEX: return "inconsistent cube_count or sel_idx entry";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,255 @@
+"""Python binding of libvsa (the C ABI in include/vsa.h).
+
+Argument marshalling only: every function forwards torch tensors' device
+pointers and the current CUDA stream to the C entry point of the same name and
+raises ``VsaError`` on a non-zero status.  Every step of the path runs in the
+library's CUDA kernels; there is no fallback.  Importing this module loads
+``libvsa.so`` and raises if it has not been built
+(``python -m video_dit_block_vsa_b200.build``).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvsa.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build the CUDA library first "
+        "(python -m video_dit_block_vsa_b200.build)")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+VSA_OK = 0
+VSA_ERR_INVALID_ARG = 1
+VSA_ERR_UNSUPPORTED = 2
+VSA_ERR_CUDA = 3
+VSA_ERR_TIMEOUT = 4
+VSA_ERR_BAD_INDEX = 5
+
+EXPORTED = ("vsa_num_cubes", "vsa_topk_from_ratio", "vsa_workspace_bytes", "vsa_tile_permute",
+            "vsa_coarse_select", "vsa_block_sparse_fwd", "vsa_combine", "vsa_untile",
+            "vsa_get_status", "vsa_debug_wait_timeout", "vsa_strerror")
+
+
+class VsaShape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("grid_t", ctypes.c_int), ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int),
+                ("cube_t", ctypes.c_int), ("cube_h", ctypes.c_int), ("cube_w", ctypes.c_int)]
+
+
+class VsaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {vsa_strerror(code)} (code {code})")
+
+
+_P = ctypes.c_void_p
+_SP = ctypes.POINTER(VsaShape)
+_sig = {
+    "vsa_num_cubes": (ctypes.c_int, [_SP, ctypes.POINTER(ctypes.c_int)]),
+    "vsa_topk_from_ratio": (ctypes.c_int, [ctypes.c_int, ctypes.c_float, ctypes.POINTER(ctypes.c_int)]),
+    "vsa_workspace_bytes": (ctypes.c_size_t, [_SP, ctypes.c_int]),
+    "vsa_tile_permute": (ctypes.c_int, [_SP, _P, _P, _P, _P]),
+    "vsa_coarse_select": (ctypes.c_int, [_SP, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P, _P,
+                                         ctypes.c_size_t, _P]),
+    "vsa_block_sparse_fwd": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P]),
+    "vsa_combine": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P]),
+    "vsa_untile": (ctypes.c_int, [_SP, _P, _P, _P]),
+    "vsa_get_status": (ctypes.c_int, [_P]),
+    "vsa_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
+    "vsa_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+}
+for _name, (_res, _args) in _sig.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+def vsa_strerror(code: int) -> str:
+    return _lib.vsa_strerror(code).decode()
+
+
+def make_shape(batch, heads, head_dim, grid, cube=(4, 4, 4)) -> VsaShape:
+    return VsaShape(batch, heads, head_dim, grid[0], grid[1], grid[2], *cube)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != VSA_OK:
+        raise VsaError(rc, where)
+
+
+def _expect(t, dtype, shape, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+
+
+# --------------------------------------------------------------------------
+# host-only helpers
+# --------------------------------------------------------------------------
+
+def vsa_num_cubes(shape: VsaShape) -> int:
+    c = ctypes.c_int(0)
+    _check(_lib.vsa_num_cubes(ctypes.byref(shape), ctypes.byref(c)), "vsa_num_cubes")
+    return c.value
+
+
+def vsa_topk_from_ratio(num_cubes: int, ratio: float) -> int:
+    k = ctypes.c_int(0)
+    _check(_lib.vsa_topk_from_ratio(num_cubes, ratio, ctypes.byref(k)), "vsa_topk_from_ratio")
+    return k.value
+
+
+def vsa_workspace_bytes(shape: VsaShape, topk: int) -> int:
+    return int(_lib.vsa_workspace_bytes(ctypes.byref(shape), topk))
+
+
+# --------------------------------------------------------------------------
+# the five calls of the path (device tensors)
+# --------------------------------------------------------------------------
+
+def _dims(shape: VsaShape):
+    C = vsa_num_cubes(shape)
+    N = shape.grid_t * shape.grid_h * shape.grid_w
+    return shape.batch, shape.heads, N, shape.head_dim, C
+
+
+def vsa_tile_permute(shape, x, x_tiled, cube_count=None, stream=None):
+    B, H, N, d, C = _dims(shape)
+    _expect(x, torch.bfloat16, (B, H, N, d), "x")
+    _expect(x_tiled, torch.bfloat16, (B, H, 64 * C, d), "x_tiled")
+    if cube_count is not None:
+        _expect(cube_count, torch.int32, (C,), "cube_count")
+    _check(_lib.vsa_tile_permute(ctypes.byref(shape), _ptr(x), _ptr(x_tiled), _ptr(cube_count),
+                                 _stream(stream)), "vsa_tile_permute")
+
+
+def vsa_coarse_select(shape, q_tiled, k_tiled, v_tiled, cube_count, topk, sel_idx, workspace,
+                      o_coarse=None, coarse_logits=None, stream=None):
+    B, H, N, d, C = _dims(shape)
+    for n, t in (("q_tiled", q_tiled), ("k_tiled", k_tiled), ("v_tiled", v_tiled)):
+        _expect(t, torch.bfloat16, (B, H, 64 * C, d), n)
+    _expect(cube_count, torch.int32, (C,), "cube_count")
+    _expect(sel_idx, torch.int32, (B, H, C, topk), "sel_idx")
+    if o_coarse is not None:
+        _expect(o_coarse, torch.float32, (B, H, C, d), "o_coarse")
+    if coarse_logits is not None:
+        _expect(coarse_logits, torch.float32, (B, H, C, C), "coarse_logits")
+    _check(_lib.vsa_coarse_select(ctypes.byref(shape), _ptr(q_tiled), _ptr(k_tiled), _ptr(v_tiled),
+                                  _ptr(cube_count), topk, _ptr(o_coarse), _ptr(sel_idx),
+                                  _ptr(coarse_logits), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)),
+           "vsa_coarse_select")
+
+
+def vsa_block_sparse_fwd(shape, q_tiled, k_tiled, v_tiled, cube_count, sel_idx, topk,
+                         o_fine_tiled, lse=None, stream=None):
+    B, H, N, d, C = _dims(shape)
+    for n, t in (("q_tiled", q_tiled), ("k_tiled", k_tiled), ("v_tiled", v_tiled),
+                 ("o_fine_tiled", o_fine_tiled)):
+        _expect(t, torch.bfloat16, (B, H, 64 * C, d), n)
+    _expect(cube_count, torch.int32, (C,), "cube_count")
+    _expect(sel_idx, torch.int32, (B, H, C, topk), "sel_idx")
+    if lse is not None:
+        _expect(lse, torch.float32, (B, H, 64 * C), "lse")
+    _check(_lib.vsa_block_sparse_fwd(ctypes.byref(shape), _ptr(q_tiled), _ptr(k_tiled),
+                                     _ptr(v_tiled), _ptr(cube_count), _ptr(sel_idx), topk,
+                                     _ptr(o_fine_tiled), _ptr(lse), _stream(stream)),
+           "vsa_block_sparse_fwd")
+
+
+def vsa_combine(shape, o_fine_tiled, out_tiled, o_coarse=None, g_fine=None, g_coarse=None,
+                stream=None):
+    B, H, N, d, C = _dims(shape)
+    _expect(o_fine_tiled, torch.bfloat16, (B, H, 64 * C, d), "o_fine_tiled")
+    _expect(out_tiled, torch.bfloat16, (B, H, 64 * C, d), "out_tiled")
+    if g_fine is not None:
+        _expect(g_fine, torch.float32, (B, H, N), "g_fine")
+        _expect(g_coarse, torch.float32, (B, H, N), "g_coarse")
+        _expect(o_coarse, torch.float32, (B, H, C, d), "o_coarse")
+    _check(_lib.vsa_combine(ctypes.byref(shape), _ptr(o_fine_tiled), _ptr(o_coarse),
+                            _ptr(g_fine), _ptr(g_coarse), _ptr(out_tiled), _stream(stream)),
+           "vsa_combine")
+
+
+def vsa_untile(shape, x_tiled, x, stream=None):
+    B, H, N, d, C = _dims(shape)
+    _expect(x_tiled, torch.bfloat16, (B, H, 64 * C, d), "x_tiled")
+    _expect(x, torch.bfloat16, (B, H, N, d), "x")
+    _check(_lib.vsa_untile(ctypes.byref(shape), _ptr(x_tiled), _ptr(x), _stream(stream)),
+           "vsa_untile")
+
+
+def vsa_get_status(stream=None) -> int:
+    return int(_lib.vsa_get_status(_stream(stream)))
+
+
+def vsa_debug_wait_timeout(timeout_ns: int, stream=None):
+    _check(_lib.vsa_debug_wait_timeout(timeout_ns, _stream(stream)), "vsa_debug_wait_timeout")
+
+
+# --------------------------------------------------------------------------
+# convenience: the whole path with torch-allocated buffers
+# --------------------------------------------------------------------------
+
+class VsaBuffers:
+    """Device buffers for one shape and k, allocated once with torch."""
+
+    def __init__(self, shape: VsaShape, topk: int, device="cuda", want_coarse=True, want_lse=False):
+        B, H, N, d, C = _dims(shape)
+        self.shape, self.topk = shape, topk
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.q_t = torch.empty(B, H, 64 * C, d, **bf)
+        self.k_t = torch.empty(B, H, 64 * C, d, **bf)
+        self.v_t = torch.empty(B, H, 64 * C, d, **bf)
+        self.o_f = torch.empty(B, H, 64 * C, d, **bf)
+        self.out_t = torch.empty(B, H, 64 * C, d, **bf)
+        self.counts = torch.empty(C, dtype=torch.int32, device=device)
+        self.sel = torch.empty(B, H, C, topk, dtype=torch.int32, device=device)
+        self.o_c = torch.empty(B, H, C, d, dtype=torch.float32, device=device) if want_coarse else None
+        self.lse = torch.empty(B, H, 64 * C, dtype=torch.float32, device=device) if want_lse else None
+        ws = vsa_workspace_bytes(shape, topk)
+        self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
+
+
+def vsa_forward(shape, q, k, v, topk, out, g_fine=None, g_coarse=None, bufs=None, stream=None):
+    """Runs the whole path: tile q/k/v, coarse select, fine attention,
+    combine, untile into ``out`` ([B, H, N, d] bf16).  Returns the buffers."""
+    if bufs is None:
+        bufs = VsaBuffers(shape, topk, device=q.device, want_coarse=g_fine is not None)
+    vsa_tile_permute(shape, q, bufs.q_t, bufs.counts, stream)
+    vsa_tile_permute(shape, k, bufs.k_t, None, stream)
+    vsa_tile_permute(shape, v, bufs.v_t, None, stream)
+    vsa_coarse_select(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, topk, bufs.sel,
+                      bufs.workspace, o_coarse=bufs.o_c, stream=stream)
+    vsa_block_sparse_fwd(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, bufs.sel, topk,
+                         bufs.o_f, bufs.lse, stream)
+    if g_fine is not None:
+        vsa_combine(shape, bufs.o_f, bufs.out_t, bufs.o_c, g_fine, g_coarse, stream)
+        vsa_untile(shape, bufs.out_t, out, stream)
+    else:
+        vsa_untile(shape, bufs.o_f, out, stream)
+    return bufs
