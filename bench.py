@@ -374,7 +374,7 @@ def run_gpu(args, w):
 
 # Revision tag of the fine kernel; ncu traffic figures are only reported for
 # the revision they were captured on.
-KERNEL_REV = "fine-v0"
+KERNEL_REV = "fine-v1"
 
 
 def main():

@@ -21,7 +21,7 @@ cudaError_t launch_coarse_select(const Geom&, const void*, const void*, const vo
                                  cudaStream_t);
 cudaError_t launch_block_sparse_fwd(const Geom&, const CUtensorMap&, const CUtensorMap&,
                                     const CUtensorMap&, const int32_t*, const int32_t*, int,
-                                    void*, float*, int*, cudaStream_t);
+                                    void*, float*, int*, int, cudaStream_t);
 cudaError_t launch_debug_wait(uint64_t, int*, cudaStream_t);
 
 // Device-side status word, one per device that loads the library.
@@ -252,7 +252,7 @@ int vsa_block_sparse_fwd(const vsa_shape* shape, const void* q_tiled, const void
       tiled_map(g, v_tiled, &tv) != VSA_OK)
     return VSA_ERR_CUDA;
   return cuda_rc(launch_block_sparse_fwd(g, tq, tk, tv, cube_count, sel_idx, topk, o_fine_tiled,
-                                         lse, st->status, stream));
+                                         lse, st->status, st->sms, stream));
 }
 
 int vsa_get_status(cudaStream_t stream) {

@@ -3,19 +3,32 @@
 // 5 秒即生一个 5 秒视频", section "一张卡，秒生视频": the fine block-sparse
 // kernel over a 64x64 block mask).
 //
-// One CTA per (query cube, b*h); 4 warps.  Tiles move by TMA (128-byte
-// swizzle) into shared memory; S = Q K^T and O += P V run on the tcgen05
-// tensor cores (M = 64 rows, bf16 operands, float32 accumulators in TMEM);
-// the online softmax reads S from TMEM (one query row per thread), writes
-// P as bf16 into a swizzled smem tile for the second MMA and rescales O in
-// TMEM when the running row maximum grows.
-//
-// TMEM layout for M = 64 (cta_group::1): row m of a 64-row accumulator sits
-// in lane (m % 16) + 32 * (m / 16), i.e. lanes 0..15 of each warp's
-// 32-lane sub-partition; thread `lane < 16` of warp w owns row 16w + lane.
-//
-// Every wait is bounded (4 s of wall time); on a timeout the CTA records
-// VSA_ERR_TIMEOUT, skips the remaining work, frees its TMEM and exits.
+// Design (sm_100a):
+//  * Persistent CTAs, one per SM, walk work items head-major; an item is a
+//    pair of query cubes (A, B) of one (b, h).  Each cube has its own key
+//    list, so every MMA has M = 64 rows (one cube); the two cubes ping-pong
+//    so that the tensor core works on one while the other's softmax runs.
+//  * Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (one thread),
+//    warps 4-7 = softmax of cube A, warps 8-11 = softmax of cube B.
+//  * A "step" covers two selected key cubes (128 keys, one N = 128 MMA;
+//    an odd k ends with a 64-key step).  Keys and values stream through a
+//    ring of 128-key smem slots (128-byte swizzle, TMA-filled) in exactly the
+//    order the MMA issuer consumes them: K_A0 K_B0 | V_A0 K_A1 V_B0 K_B1 | ...
+//  * TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+d),
+//    O_B [256+d, 256+2d).  The softmax writes P (bf16 pairs) over the first 64
+//    columns of its S, and O += P V reads P straight from TMEM (A operand in
+//    TMEM), so P never touches shared memory.  MMAs issued by one thread
+//    execute in order, so the next S = Q K^T cannot overwrite P before the
+//    P V that reads it.
+//  * M = 64 accumulators use TMEM lanes 0-15 of each warp's 32-lane
+//    sub-partition; the softmax reads them with the 16-lane .16x32bx2 shape:
+//    thread t holds row 16*(warp%4) + t%16, columns [64*(t/16), +64) of the
+//    step, i.e. exactly one key cube's 64 keys.
+//  * Online softmax in log2 units with conditional rescaling: the running
+//    reference max only moves (and O, l are rescaled) when a row's max grows
+//    by more than 2^8, so most steps skip the O round trip through registers.
+//  * Every wait is bounded (4 s); on a timeout the CTA records
+//    VSA_ERR_TIMEOUT, every role stops, TMEM is freed and the CTA exits.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -27,53 +40,389 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 128;
-constexpr uint32_t kHalfTile = 64 * 128;  // one [64 rows x 64 bf16] swizzled half tile, bytes
-constexpr uint32_t kTmemCols = 256;       // S: cols [0, 64); O: cols [128, 128 + d)
-constexpr uint32_t kColO = 128;
+constexpr int kWarps = 12;
+constexpr int kThreads = kWarps * 32;
+constexpr int kProducerWarp = 0;
+constexpr int kMmaWarp = 1;
+constexpr int kSoftmaxWarp0 = 4;  // warps 4..7: cube A, 8..11: cube B
+constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleLog2 = 8.0f;  // rescale only when a row max grows by > 2^8
+
+template <int D>
+struct Cfg {
+  static constexpr int kHalves = D / 64;                       // 128-byte atoms per row
+  static constexpr uint32_t kQHalf = 64 * 128;                 // [64 rows x 128 B]
+  static constexpr uint32_t kQBytes = kHalves * kQHalf;        // one query cube tile
+  static constexpr uint32_t kKVHalf = 128 * 128;               // [128 rows x 128 B]
+  static constexpr uint32_t kSlotBytes = kHalves * kKVHalf;    // 128 keys x D
+  static constexpr int kSlots = D == 128 ? 5 : 10;
+  static constexpr uint32_t kRingOff = 4 * kQBytes;            // Q: 2 items x 2 cubes
+  static constexpr uint32_t kBarOff = kRingOff + kSlots * kSlotBytes;
+  static constexpr size_t kSmem = 1024 + kBarOff + 320;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128;
+  static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(64, D, false, true);  // P (TMEM), V MN-major
+};
+
+struct Shared {
+  uint64_t* q_full;
+  uint64_t* q_empty;
+  uint64_t* kv_full;
+  uint64_t* kv_empty;
+  uint64_t* s_full;
+  uint64_t* p_full;
+  uint64_t* o_full;
+  volatile int* abort_flag;
+  uint8_t* base;
+};
+
+struct Item {
+  int bh, i0, i1, row0;
+  bool has_b;
+};
+
+__device__ __forceinline__ Item decode(const Geom& g, int item, int pairs) {
+  Item it;
+  it.bh = item / pairs;
+  const int pr = item - it.bh * pairs;
+  it.i0 = 2 * pr;
+  it.i1 = it.i0 + 1;
+  it.has_b = it.i1 < g.C;
+  it.row0 = it.bh * static_cast<int>(g.rows);
+  return it;
+}
+
+__device__ __forceinline__ void fail(const Shared& sh, int* status) {
+  report(status, VSA_ERR_TIMEOUT);
+  *sh.abort_flag = 1;
+}
 
 __device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
   const __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&p);
 }
 
+// ------------------------------------------------------------------ producer
 template <int D>
-__global__ void __launch_bounds__(kThreads) fine_fwd_kernel(
+__device__ void producer(const Shared& sh, const Geom& g, const CUtensorMap* tq,
+                         const CUtensorMap* tk, const CUtensorMap* tv,
+                         const int32_t* __restrict__ counts, const int32_t* __restrict__ sel,
+                         int topk, int* status) {
+  using Cf = Cfg<D>;
+  const int pairs = (g.C + 1) / 2;
+  const int items = g.B * g.H * pairs;
+  const int nsteps = (topk + 1) / 2;
+  uint32_t ring = 0;
+  int t = 0;
+  for (int item = blockIdx.x; item < items; item += gridDim.x, ++t) {
+    if (*sh.abort_flag) return;
+    const Item it = decode(g, item, pairs);
+    if (__ldg(&counts[it.i0]) != cube_valid(g, it.i0) ||
+        (it.has_b && __ldg(&counts[it.i1]) != cube_valid(g, it.i1)))
+      report(status, VSA_ERR_BAD_INDEX);
+    // ---- query tiles of both cubes
+    const int qb = t & 1;
+    if (!mbar_wait(&sh.q_empty[qb], ((t >> 1) & 1) ^ 1)) return fail(sh, status);
+    mbar_arrive_expect_tx(&sh.q_full[qb], (it.has_b ? 2 : 1) * Cf::kQBytes);
+    uint8_t* qdst = sh.base + qb * 2 * Cf::kQBytes;
+#pragma unroll
+    for (int h = 0; h < Cf::kHalves; ++h) {
+      tma_load_2d(qdst + h * Cf::kQHalf, tq, &sh.q_full[qb], h * 64, it.row0 + it.i0 * 64);
+      if (it.has_b)
+        tma_load_2d(qdst + Cf::kQBytes + h * Cf::kQHalf, tq, &sh.q_full[qb], h * 64,
+                    it.row0 + it.i1 * 64);
+    }
+    // ---- key / value slots, in the MMA issuer's order
+    const int32_t* list0 = sel + (static_cast<long long>(it.bh) * g.C + it.i0) * topk;
+    const int32_t* list1 = list0 + topk;
+    int prev0 = -1, prev1 = -1;
+    auto load = [&](int c, int j, bool is_v) -> bool {
+      const int slot = static_cast<int>(ring % Cf::kSlots);
+      const uint32_t round = ring / Cf::kSlots;
+      ++ring;
+      if (!mbar_wait(&sh.kv_empty[slot], (round & 1u) ^ 1u)) return false;
+      const int a = 2 * j;
+      const int nk = (a + 1 < topk) ? 2 : 1;
+      mbar_arrive_expect_tx(&sh.kv_full[slot], nk * 64 * D * 2);
+      uint8_t* dst = sh.base + Cf::kRingOff + slot * Cf::kSlotBytes;
+      const int32_t* list = c == 0 ? list0 : list1;
+      int& prev = c == 0 ? prev0 : prev1;
+      for (int r = 0; r < nk; ++r) {
+        int jr = __ldg(&list[a + r]);
+        if (!is_v) {  // validate once per index (on the key load)
+          if (jr < 0 || jr >= g.C || jr <= prev) report(status, VSA_ERR_BAD_INDEX);
+          prev = jr;
+        }
+        jr = jr < 0 ? 0 : (jr >= g.C ? g.C - 1 : jr);
+#pragma unroll
+        for (int h = 0; h < Cf::kHalves; ++h)
+          tma_load_2d(dst + h * Cf::kKVHalf + r * (64 * 128), is_v ? tv : tk, &sh.kv_full[slot],
+                      h * 64, it.row0 + jr * 64);
+      }
+      return true;
+    };
+    if (!load(0, 0, false)) return fail(sh, status);
+    if (it.has_b && !load(1, 0, false)) return fail(sh, status);
+    for (int j = 0; j < nsteps; ++j) {
+      if (*sh.abort_flag) return;
+      if (!load(0, j, true)) return fail(sh, status);
+      if (j + 1 < nsteps && !load(0, j + 1, false)) return fail(sh, status);
+      if (it.has_b) {
+        if (!load(1, j, true)) return fail(sh, status);
+        if (j + 1 < nsteps && !load(1, j + 1, false)) return fail(sh, status);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ MMA issuer
+template <int D>
+__device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int topk,
+                           int* status) {
+  using Cf = Cfg<D>;
+  const int pairs = (g.C + 1) / 2;
+  const int items = g.B * g.H * pairs;
+  const int nsteps = (topk + 1) / 2;
+  uint32_t ring = 0;
+  uint32_t p_phase0 = 0u, p_phase1 = 0u;
+  int t = 0;
+  for (int item = blockIdx.x; item < items; item += gridDim.x, ++t) {
+    if (*sh.abort_flag) return;
+    const Item it = decode(g, item, pairs);
+    const int qb = t & 1;
+    if (!mbar_wait(&sh.q_full[qb], (t >> 1) & 1)) return fail(sh, status);
+    tc_fence_after();
+    const uint32_t qa0 = smem_u32(sh.base + qb * 2 * Cf::kQBytes);
+    const uint32_t qa1 = qa0 + Cf::kQBytes;
+    auto next_slot = [&](int& slot) -> bool {
+      slot = static_cast<int>(ring % Cf::kSlots);
+      const uint32_t round = ring / Cf::kSlots;
+      ++ring;
+      if (!mbar_wait(&sh.kv_full[slot], round & 1u)) return false;
+      tc_fence_after();
+      return true;
+    };
+    // S_c = Q_c K^T over one step's keys
+    auto qk = [&](int c, int j) -> bool {
+      int slot;
+      if (!next_slot(slot)) return false;
+      const int nk = (2 * j + 1 < topk) ? 2 : 1;
+      const uint32_t idesc = idesc_bf16_f32(64, 64 * nk, false, false);
+      const uint32_t kb = smem_u32(sh.base + Cf::kRingOff + slot * Cf::kSlotBytes);
+      const uint32_t qa = c == 0 ? qa0 : qa1;
+      const uint32_t dS = tmem + (c == 0 ? Cf::kColS0 : Cf::kColS1);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t ao = (kk >> 2) * Cf::kQHalf + (kk & 3) * 32;
+        const uint32_t bo = (kk >> 2) * Cf::kKVHalf + (kk & 3) * 32;
+        umma_ss(dS, sdesc_sw128(qa + ao, 16, 1024), sdesc_sw128(kb + bo, 16, 1024), idesc,
+                kk > 0 ? 1u : 0u);
+      }
+      umma_commit(&sh.kv_empty[slot]);
+      umma_commit(&sh.s_full[c]);
+      return true;
+    };
+    // O_c += P_c V over one step's keys; P_c read from TMEM
+    auto pv = [&](int c, int j) -> bool {
+      uint32_t& ph = c == 0 ? p_phase0 : p_phase1;
+      if (!mbar_wait(&sh.p_full[c], ph)) return false;
+      ph ^= 1u;
+      tc_fence_after();
+      int slot;
+      if (!next_slot(slot)) return false;
+      const int ksteps = ((2 * j + 1 < topk) ? 2 : 1) * 4;  // 16 keys per MMA
+      const uint32_t vb = smem_u32(sh.base + Cf::kRingOff + slot * Cf::kSlotBytes);
+      const uint32_t dO = tmem + (c == 0 ? Cf::kColO0 : Cf::kColO1);
+      const uint32_t aP = tmem + (c == 0 ? Cf::kColS0 : Cf::kColS1);
+      for (int kk = 0; kk < ksteps; ++kk) {
+        umma_ts(dO, aP + kk * 8, sdesc_sw128(vb + kk * 2048, Cf::kKVHalf, 1024), Cf::kIdescPV,
+                (j > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(&sh.kv_empty[slot]);
+      if (j == nsteps - 1) umma_commit(&sh.o_full[c]);
+      return true;
+    };
+    if (!qk(0, 0)) return fail(sh, status);
+    if (it.has_b && !qk(1, 0)) return fail(sh, status);
+    for (int j = 0; j < nsteps; ++j) {
+      if (*sh.abort_flag) return;
+      if (!pv(0, j)) return fail(sh, status);
+      if (j + 1 < nsteps && !qk(0, j + 1)) return fail(sh, status);
+      if (it.has_b) {
+        if (!pv(1, j)) return fail(sh, status);
+        if (j + 1 < nsteps && !qk(1, j + 1)) return fail(sh, status);
+      }
+    }
+    umma_commit(&sh.q_empty[qb]);  // Q buffer free once this item's MMAs complete
+  }
+}
+
+// ------------------------------------------------------------------ softmax
+template <int D>
+__device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c,
+                           const int32_t* __restrict__ sel, int topk,
+                           __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+                           int* status) {
+  using Cf = Cfg<D>;
+  constexpr int kOH = D / 2;  // O columns per thread (half a row)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wq = warp & 3;              // TMEM sub-partition of this warp
+  const int hh = lane >> 4;             // which 64-key half of a step this thread holds
+  const int r = wq * 16 + (lane & 15);  // query row of the cube
+  const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
+  const uint32_t tS = tmem + lane_addr + (c == 0 ? Cf::kColS0 : Cf::kColS1);
+  const uint32_t tO = tmem + lane_addr + (c == 0 ? Cf::kColO0 : Cf::kColO1);
+  const float sl2 = kLog2e * rsqrtf(static_cast<float>(D));
+  const int pairs = (g.C + 1) / 2;
+  const int items = g.B * g.H * pairs;
+  const int nsteps = (topk + 1) / 2;
+  uint32_t s_phase = 0u, o_phase = 0u;
+
+  for (int item = blockIdx.x; item < items; item += gridDim.x) {
+    if (*sh.abort_flag) return;
+    const Item it = decode(g, item, pairs);
+    if (c == 1 && !it.has_b) continue;
+    const int i = c == 0 ? it.i0 : it.i1;
+    const int ni = cube_valid(g, i);
+    const int32_t* list = sel + (static_cast<long long>(it.bh) * g.C + i) * topk;
+    float m_ref = -INFINITY, l_part = 0.f;
+    for (int j = 0; j < nsteps; ++j) {
+      const int a = 2 * j + hh;
+      int nh = 0;
+      if (a < topk) {
+        int jr = __ldg(&list[a]);
+        jr = jr < 0 ? 0 : (jr >= g.C ? g.C - 1 : jr);
+        nh = cube_valid(g, jr);
+      }
+      if (!mbar_wait(&sh.s_full[c], s_phase)) return fail(sh, status);
+      s_phase ^= 1u;
+      tc_fence_after();
+      uint32_t sv[64];
+      tmem_ld_16x32bx2_x64(tS, sv);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        const float x = e < nh ? __uint_as_float(sv[e]) : -INFINITY;
+        sv[e] = __float_as_uint(x);
+        mx = fmaxf(mx, x);
+      }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float mx2 = mx * sl2;
+      float alpha = 1.f;
+      bool need = false;
+      if (j == 0) {
+        m_ref = mx2;
+      } else if (mx2 > m_ref + kRescaleLog2) {
+        alpha = exp2f(m_ref - mx2);
+        m_ref = mx2;
+        need = true;
+      }
+      if (__any_sync(0xffffffffu, need)) {  // the previous P V has completed
+        uint32_t ov[kOH];
+        if constexpr (kOH == 64) {
+          tmem_ld_16x32bx2_x64(tO, ov);
+        } else {
+          tmem_ld_16x32bx2_x32(tO, ov);
+        }
+#pragma unroll
+        for (int e = 0; e < kOH; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+        if constexpr (kOH == 64) {
+          tmem_st_16x32bx2_x64(tO, ov);
+        } else {
+          tmem_st_16x32bx2_x32(tO, ov);
+        }
+      }
+      l_part *= alpha;
+      float sum = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const float p0 = exp2f(fmaf(__uint_as_float(sv[2 * e]), sl2, -m_ref));
+        const float p1 = exp2f(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -m_ref));
+        sum += p0 + p1;
+        pk[e] = pack2_bf16(p0, p1);
+      }
+      l_part += sum;
+      tmem_st_16x32bx2_x32(tS, pk);  // P over the first 64 columns of S
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sh.p_full[c]);
+    }
+    // ---- epilogue: O / l -> bf16; pad rows -> 0
+    if (!mbar_wait(&sh.o_full[c], o_phase)) return fail(sh, status);
+    o_phase ^= 1u;
+    tc_fence_after();
+    uint32_t ov[kOH];
+    if constexpr (kOH == 64) {
+      tmem_ld_16x32bx2_x64(tO, ov);
+    } else {
+      tmem_ld_16x32bx2_x32(tO, ov);
+    }
+    const float l = l_part + __shfl_xor_sync(0xffffffffu, l_part, 16);
+    const bool valid = r < ni;
+    const float inv = 1.0f / l;
+    uint4* orow = reinterpret_cast<uint4*>(
+        out + (static_cast<long long>(it.row0) + i * 64 + r) * D + hh * kOH);
+#pragma unroll
+    for (int q8 = 0; q8 < kOH / 8; ++q8) {
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (valid) {
+        w.x = pack2_bf16(__uint_as_float(ov[q8 * 8 + 0]) * inv, __uint_as_float(ov[q8 * 8 + 1]) * inv);
+        w.y = pack2_bf16(__uint_as_float(ov[q8 * 8 + 2]) * inv, __uint_as_float(ov[q8 * 8 + 3]) * inv);
+        w.z = pack2_bf16(__uint_as_float(ov[q8 * 8 + 4]) * inv, __uint_as_float(ov[q8 * 8 + 5]) * inv);
+        w.w = pack2_bf16(__uint_as_float(ov[q8 * 8 + 6]) * inv, __uint_as_float(ov[q8 * 8 + 7]) * inv);
+      }
+      orow[q8] = w;
+    }
+    if (lse != nullptr && hh == 0)
+      lse[static_cast<long long>(it.row0) + i * 64 + r] =
+          valid ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) fine_fwd_kernel(
     const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
     const __grid_constant__ CUtensorMap tv, Geom g, const int32_t* __restrict__ counts,
     const int32_t* __restrict__ sel, int topk, __nv_bfloat16* __restrict__ out,
     float* __restrict__ lse, int* status) {
-  constexpr int kHalves = D / 64;
-  constexpr uint32_t kTile = kHalves * kHalfTile;
-  constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 64, false, false);  // Q K-major, K K-major
-  constexpr uint32_t kIdescPV = idesc_bf16_f32(64, D, false, true);    // P K-major, V MN-major
-
+  using Cf = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* Qs = smem;
-  uint8_t* Ks = Qs + kTile;
-  uint8_t* Vs = Ks + kTile;
-  uint8_t* Ps = Vs + kTile;  // [64 rows x 64 keys] bf16, one half tile
-  uint64_t* bars = reinterpret_cast<uint64_t*>(Ps + kHalfTile);  // q, kv, mma
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cf::kBarOff);
+  Shared sh;
+  sh.base = smem;
+  sh.q_full = bars;
+  sh.q_empty = bars + 2;
+  sh.kv_full = bars + 4;
+  sh.kv_empty = bars + 4 + Cf::kSlots;
+  sh.s_full = bars + 4 + 2 * Cf::kSlots;
+  sh.p_full = sh.s_full + 2;
+  sh.o_full = sh.s_full + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sh.o_full + 2);
+  sh.abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int i = blockIdx.x;
-  const int bh = blockIdx.y;
-  const int row = warp * 16 + lane;  // query row owned by this thread (lane < 16)
-  const bool has_row = lane < 16;
-
-  if (warp == 0) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (tid == 32) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
-    mbar_init(&bars[2], 1);
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&sh.q_full[q], 1);
+      mbar_init(&sh.q_empty[q], 1);
+      mbar_init(&sh.s_full[q], 1);
+      mbar_init(&sh.p_full[q], 128);
+      mbar_init(&sh.o_full[q], 1);
+    }
+    for (int s = 0; s < Cf::kSlots; ++s) {
+      mbar_init(&sh.kv_full[s], 1);
+      mbar_init(&sh.kv_empty[s], 1);
+    }
+    *sh.abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tq);
     prefetch_tmap(&tk);
@@ -83,188 +432,30 @@ __global__ void __launch_bounds__(kThreads) fine_fwd_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t tS = tmem + lane_off;
-  const uint32_t tO = tmem + lane_off + kColO;
 
-  const int row0 = bh * static_cast<int>(g.rows);  // first tiled row of this (b, h)
-  const int ni = cube_valid(g, i);
-  if (tid == 0 && counts[i] != ni) report(status, VSA_ERR_BAD_INDEX);
-  const int32_t* my_sel = sel + (static_cast<long long>(bh) * g.C + i) * topk;
-
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bars[0], kTile);
-#pragma unroll
-    for (int h = 0; h < kHalves; ++h) tma_load_2d(Qs + h * kHalfTile, &tq, &bars[0], h * 64, row0 + i * 64);
-  }
-  bool timed_out = !mbar_wait(&bars[0], 0);
-
-  const float sl2 = kLog2e / sqrtf(static_cast<float>(D));  // scores -> log2 units
-  float m_run = -INFINITY, l_run = 0.f;
-  uint32_t kv_phase = 0, mma_phase = 0;
-  int prev = -1;
-
-  for (int jj = 0; jj < topk && !__syncthreads_or(timed_out); ++jj) {
-    int j = __ldg(&my_sel[jj]);
-    if (j < 0 || j >= g.C || j <= prev) {
-      if (tid == 0) report(status, VSA_ERR_BAD_INDEX);
-      j = j < 0 ? 0 : (j >= g.C ? g.C - 1 : j);
-    }
-    prev = j;
-    const int nj = cube_valid(g, j);
-
-    // ---- K_j, V_j -> smem
-    if (tid == 0) {
-      mbar_arrive_expect_tx(&bars[1], 2 * kTile);
-#pragma unroll
-      for (int h = 0; h < kHalves; ++h) {
-        tma_load_2d(Ks + h * kHalfTile, &tk, &bars[1], h * 64, row0 + j * 64);
-        tma_load_2d(Vs + h * kHalfTile, &tv, &bars[1], h * 64, row0 + j * 64);
-      }
-    }
-    timed_out |= !mbar_wait(&bars[1], kv_phase);
-    kv_phase ^= 1u;
-    if (__syncthreads_or(timed_out)) break;
-
-    // ---- S = Q K^T  (M=64, N=64, K=D)
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t qa = smem_u32(Qs), ka = smem_u32(Ks);
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * kHalfTile + (kk & 3) * 32;
-        umma_ss(tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
-                kIdescQK, kk > 0 ? 1u : 0u);
-      }
-      umma_commit(&bars[2]);
-    }
-    timed_out |= !mbar_wait(&bars[2], mma_phase);
-    mma_phase ^= 1u;
-    if (__syncthreads_or(timed_out)) break;
-    tc_fence_after();
-
-    // ---- online softmax on this thread's row
-    float s[64];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float t[16];
-      tmem_ld16(tS + c * 16, t);
-#pragma unroll
-      for (int e = 0; e < 16; ++e) s[c * 16 + e] = t[e];
-    }
-    float mx = -INFINITY;
-#pragma unroll
-    for (int e = 0; e < 64; ++e) {
-      if (e >= nj) s[e] = -INFINITY;  // pad key slots
-      mx = fmaxf(mx, s[e]);
-    }
-    const float m_new = fmaxf(m_run, mx * sl2);
-    const float alpha = exp2f(m_run - m_new);
-    float sum = 0.f;
-#pragma unroll
-    for (int e = 0; e < 64; ++e) {
-      s[e] = exp2f(fmaf(s[e], sl2, -m_new));
-      sum += s[e];
-    }
-    l_run = l_run * alpha + sum;
-    m_run = m_new;
-    if (has_row) {
-      uint8_t* prow = Ps + row * 128;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 w;
-        w.x = pack2_bf16(s[8 * c + 0], s[8 * c + 1]);
-        w.y = pack2_bf16(s[8 * c + 2], s[8 * c + 3]);
-        w.z = pack2_bf16(s[8 * c + 4], s[8 * c + 5]);
-        w.w = pack2_bf16(s[8 * c + 6], s[8 * c + 7]);
-        *reinterpret_cast<uint4*>(prow + ((c ^ (row & 7)) << 4)) = w;
-      }
-    }
-    if (jj > 0) {  // O *= alpha before accumulating this block
-#pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        float o[16];
-        tmem_ld16(tO + c * 16, o);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) o[e] *= alpha;
-        tmem_st16(tO + c * 16, o);
-      }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- O += P V  (M=64, N=D, K=64)
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t pa = smem_u32(Ps), va = smem_u32(Vs);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        umma_ss(tmem + kColO, sdesc_sw128(pa + kk * 32, 16, 1024),
-                sdesc_sw128(va + kk * 2048, kHalfTile, 1024), kIdescPV,
-                (jj > 0 || kk > 0) ? 1u : 0u);
-      }
-      umma_commit(&bars[2]);
-    }
-    timed_out |= !mbar_wait(&bars[2], mma_phase);
-    mma_phase ^= 1u;
-    tc_fence_after();
-  }
-
-  if (__syncthreads_or(timed_out)) {
-    if (tid == 0) report(status, VSA_ERR_TIMEOUT);
-  } else {
-    // ---- epilogue: O / l -> bf16, pad rows -> 0
-    const bool valid = row < ni;
-    const float inv = valid ? 1.0f / l_run : 0.f;
-    __nv_bfloat16* orow = out + (static_cast<long long>(row0) + i * 64 + row) * D;
-#pragma unroll
-    for (int c = 0; c < D / 16; ++c) {
-      float o[16];
-      tmem_ld16(tO + c * 16, o);
-      if (!valid) {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) o[e] = 0.f;
-      }
-      if (has_row) {
-        uint4 w0, w1;
-        w0.x = pack2_bf16(o[0] * inv, o[1] * inv);
-        w0.y = pack2_bf16(o[2] * inv, o[3] * inv);
-        w0.z = pack2_bf16(o[4] * inv, o[5] * inv);
-        w0.w = pack2_bf16(o[6] * inv, o[7] * inv);
-        w1.x = pack2_bf16(o[8] * inv, o[9] * inv);
-        w1.y = pack2_bf16(o[10] * inv, o[11] * inv);
-        w1.z = pack2_bf16(o[12] * inv, o[13] * inv);
-        w1.w = pack2_bf16(o[14] * inv, o[15] * inv);
-        reinterpret_cast<uint4*>(orow + c * 16)[0] = w0;
-        reinterpret_cast<uint4*>(orow + c * 16)[1] = w1;
-      }
-    }
-    if (lse != nullptr && has_row) {
-      lse[static_cast<long long>(row0) + i * 64 + row] =
-          valid ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
-    }
+  if (warp == kProducerWarp) {
+    if (lane == 0) producer<D>(sh, g, &tq, &tk, &tv, counts, sel, topk, status);
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) mma_issuer<D>(sh, g, tmem, topk, status);
+  } else if (warp >= kSoftmaxWarp0) {
+    softmax_wg<D>(sh, g, tmem, (warp - kSoftmaxWarp0) >> 2, sel, topk, out, lse, status);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace
 
-// Shared memory request: the tiles plus alignment slack, raised to 100 KB so
-// that at most two CTAs share an SM and their TMEM (2 x 256 columns) fits.
-size_t fine_smem_bytes(int d) {
-  const size_t need = 1024 /* alignment slack */ + 3 * (d / 64) * kHalfTile + kHalfTile + 64;
-  return need > 100 * 1024 ? need : 100 * 1024;
-}
+size_t fine_smem_bytes(int d) { return d == 128 ? Cfg<128>::kSmem : Cfg<64>::kSmem; }
 
 cudaError_t launch_block_sparse_fwd(const Geom& g, const CUtensorMap& tq, const CUtensorMap& tk,
                                     const CUtensorMap& tv, const int32_t* counts,
                                     const int32_t* sel, int topk, void* out, float* lse,
-                                    int* status, cudaStream_t s) {
+                                    int* status, int sms, cudaStream_t s) {
+  const long long items = static_cast<long long>(g.B) * g.H * ((g.C + 1) / 2);
+  const int grid = static_cast<int>(items < sms ? items : sms);
   const size_t smem = fine_smem_bytes(g.d);
-  dim3 grid(static_cast<unsigned>(g.C), static_cast<unsigned>(g.B * g.H));
   cudaError_t err;
   if (g.d == 128) {
     err = cudaFuncSetAttribute(fine_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
