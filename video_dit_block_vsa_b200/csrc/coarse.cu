@@ -21,8 +21,7 @@ namespace vsa {
 namespace {
 
 constexpr int kCoarseThreads = 256;
-constexpr int kKeyChunk = 32;
-constexpr int kLogitBudgetBytes = 160 * 1024;
+constexpr int kLogitBudgetBytes = 132 * 1024;
 
 // ------------------------------------------------------------------ pooling
 // One warp per (tensor, b*h, cube).  A row of d bf16 is d/8 16-byte chunks;
@@ -148,17 +147,28 @@ __device__ void warp_topk(const float* row, int C, int k, int* hist, int32_t* ou
 }
 
 // ------------------------------------------------------------------ coarse
-// grid (ceil(C/R), B*H); R query cubes per CTA; 256 threads.
-// smem: logits [R][C] f32 | q rows [R][d] | key/value chunk [32][d+1] | hist [8][256]
+// grid (ceil(C/R), B*H), 256 threads, R <= 16 query cubes per CTA.
+// smem: S [R][Cp] f32 (Cp = C rounded up to 4) | qT [d][16] | staging
+// [32][260] (key slices, then value chunks) | hist [8][256].
+//
+// Logits: a 16-row x 256-key tile per pass; thread t owns rows 4*(t/64)..+3
+// and keys 4*(t%64)..+3 (16 accumulators), over head-dim slices of 32
+// staged transposed in smem, so each step is two 128-bit smem loads for 16
+// FMAs.  O_c: thread t owns rows 2*(t/32), +1 and d/32 columns.
+constexpr int kTileKeys = 256;
+constexpr int kSlice = 32;
+constexpr int kStagePitch = kTileKeys + 4;
+
 __global__ void __launch_bounds__(kCoarseThreads) coarse_kernel(
     Geom g, int R, int topk, const float* __restrict__ ws, float* __restrict__ o_coarse,
     int32_t* __restrict__ sel, float* __restrict__ logits_out) {
-  extern __shared__ float sm[];
-  const int C = g.C, d = g.d, dp = g.d + 1;
-  float* S = sm;                                   // [R][C]
-  float* qs = S + static_cast<size_t>(R) * C;      // [R][d]
-  float* ks = qs + static_cast<size_t>(R) * d;     // [32][d+1]
-  int* hist = reinterpret_cast<int*>(ks + kKeyChunk * dp);  // [8][256]
+  extern __shared__ __align__(16) float sm[];
+  const int C = g.C, d = g.d;
+  const int Cp = (C + 3) & ~3;
+  float* S = sm;                                     // [R][Cp]
+  float* qT = S + static_cast<size_t>(R) * Cp;       // [d][16]
+  float* stage = qT + static_cast<size_t>(d) * 16;   // [32][kStagePitch]
+  int* hist = reinterpret_cast<int*>(stage + kSlice * kStagePitch);  // [8][256]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y;
@@ -170,36 +180,65 @@ __global__ void __launch_bounds__(kCoarseThreads) coarse_kernel(
   const float* vbar = ws + 2 * plane + (static_cast<long long>(bh) * C) * d;
   const float scale = 1.0f / sqrtf(static_cast<float>(d));
 
-  for (int e = tid; e < R * d; e += kCoarseThreads) {
-    const int r = e / d;
-    qs[e] = r < rows ? qbar[static_cast<long long>(i0 + r) * d + (e - r * d)] : 0.f;
+  for (int e = tid; e < 16 * d; e += kCoarseThreads) {  // qT[col][row]
+    const int r = e & 15, col = e >> 4;
+    qT[e] = r < rows ? qbar[static_cast<long long>(i0 + r) * d + col] : 0.f;
   }
-  // ---- logits: thread -> key jj = lane of the chunk, rows warp, warp+8, ...
-  for (int j0 = 0; j0 < C; j0 += kKeyChunk) {
-    __syncthreads();
-    const int nk = min(kKeyChunk, C - j0);
-    for (int e = tid; e < kKeyChunk * d; e += kCoarseThreads) {
-      const int jj = e / d, col = e - jj * d;
-      ks[jj * dp + col] = jj < nk ? kbar[static_cast<long long>(j0 + jj) * d + col] : 0.f;
+  // ---- logits
+  const int rg = tid >> 6, kg = tid & 63;
+  for (int j0 = 0; j0 < C; j0 += kTileKeys) {
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+    for (int e0 = 0; e0 < d; e0 += kSlice) {
+      __syncthreads();
+      // stage keys j0..j0+255, dims e0..e0+31, transposed: stage[dim][key]
+      for (int idx = tid; idx < kTileKeys * (kSlice / 4); idx += kCoarseThreads) {
+        const int jj = idx >> 3, q4 = idx & 7;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j0 + jj < C)
+          v = *reinterpret_cast<const float4*>(kbar + static_cast<long long>(j0 + jj) * d + e0 + 4 * q4);
+        stage[(4 * q4 + 0) * kStagePitch + jj] = v.x;
+        stage[(4 * q4 + 1) * kStagePitch + jj] = v.y;
+        stage[(4 * q4 + 2) * kStagePitch + jj] = v.z;
+        stage[(4 * q4 + 3) * kStagePitch + jj] = v.w;
+      }
+      __syncthreads();
+#pragma unroll 8
+      for (int ee = 0; ee < kSlice; ++ee) {
+        const float4 qv = *reinterpret_cast<const float4*>(qT + (e0 + ee) * 16 + 4 * rg);
+        const float4 kv = *reinterpret_cast<const float4*>(stage + ee * kStagePitch + 4 * kg);
+        const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
+        const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(qa[a], ka[b], acc[a][b]);
+      }
     }
-    __syncthreads();
-    if (lane < nk) {
-      for (int r = warp; r < rows; r += 8) {
-        const float* qr = qs + r * d;
-        const float* kr = ks + lane * dp;
-        float acc = 0.f;
-        for (int e = 0; e < d; ++e) acc = fmaf(qr[e], kr[e], acc);
-        const float s = acc * scale;
-        S[static_cast<size_t>(r) * C + j0 + lane] = s;
-        if (logits_out != nullptr)
-          logits_out[(static_cast<long long>(bh) * C + i0 + r) * C + j0 + lane] = s;
+    const int jb = j0 + 4 * kg;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int r = 4 * rg + a;
+      if (r >= rows) continue;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int j = jb + b;
+        if (j < C) {
+          const float s = acc[a][b] * scale;
+          S[static_cast<size_t>(r) * Cp + j] = s;
+          if (logits_out != nullptr)
+            logits_out[(static_cast<long long>(bh) * C + i0 + r) * C + j] = s;
+        }
       }
     }
   }
   __syncthreads();
   // ---- top-k on the logits, then softmax in place (one warp per row)
   for (int r = warp; r < rows; r += 8) {
-    float* row = S + static_cast<size_t>(r) * C;
+    float* row = S + static_cast<size_t>(r) * Cp;
     warp_topk(row, C, topk, hist + warp * 256,
               sel + (static_cast<long long>(bh) * C + i0 + r) * topk);
     float mx = -INFINITY;
@@ -214,55 +253,74 @@ __global__ void __launch_bounds__(kCoarseThreads) coarse_kernel(
     for (int off = 16; off; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
     const float inv = 1.0f / z;
     __syncwarp();
-    for (int j = lane; j < C; j += 32) row[j] *= inv;
+    for (int j = lane; j < Cp; j += 32) row[j] = j < C ? row[j] * inv : 0.f;
   }
   if (o_coarse == nullptr) return;
-  // ---- O_c = P vbar: thread -> column e = tid % d, rows tid / d + G*m
-  const int G = kCoarseThreads / d;  // 2 (d=128) or 4 (d=64)
-  const int e = tid % d, rg = tid / d;
-  float acc[16];
-#pragma unroll
-  for (int m = 0; m < 16; ++m) acc[m] = 0.f;
-  for (int j0 = 0; j0 < C; j0 += kKeyChunk) {
+  // ---- O_c = P vbar: rows 2*(t/32), +1; columns cpt*(t%32) .. +cpt-1
+  const int cpt = d / 32;  // 4 (d=128) or 2 (d=64)
+  const int r0 = 2 * (tid >> 5), c0 = cpt * (tid & 31);
+  float o0[4] = {0.f, 0.f, 0.f, 0.f}, o1[4] = {0.f, 0.f, 0.f, 0.f};
+  const int vchunk = (kSlice * kStagePitch) / d & ~3;  // value rows per staged chunk
+  for (int j0 = 0; j0 < C; j0 += vchunk) {
     __syncthreads();
-    const int nk = min(kKeyChunk, C - j0);
-    for (int t = tid; t < kKeyChunk * d; t += kCoarseThreads) {
-      const int jj = t / d, col = t - jj * d;
-      ks[jj * dp + col] = jj < nk ? vbar[static_cast<long long>(j0 + jj) * d + col] : 0.f;
+    const int nk = min(vchunk, C - j0);
+    for (int idx = tid; idx < vchunk * d / 4; idx += kCoarseThreads) {
+      const int jj = idx / (d / 4), q4 = idx - jj * (d / 4);
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (jj < nk) v = *reinterpret_cast<const float4*>(vbar + static_cast<long long>(j0 + jj) * d + 4 * q4);
+      reinterpret_cast<float4*>(stage)[idx] = v;
     }
     __syncthreads();
-    for (int jj = 0; jj < nk; ++jj) {
-      const float vv = ks[jj * dp + e];
+    if (r0 < rows) {
+      const float* p0 = S + static_cast<size_t>(r0) * Cp + j0;
+      const float* p1 = p0 + Cp;
+      for (int jj = 0; jj < nk; jj += 4) {
+        const float4 pa = *reinterpret_cast<const float4*>(p0 + jj);
+        const float4 pb = *reinterpret_cast<const float4*>(p1 + jj);
+        const float pav[4] = {pa.x, pa.y, pa.z, pa.w};
+        const float pbv[4] = {pb.x, pb.y, pb.z, pb.w};
 #pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        const int r = rg + G * m;
-        if (r < rows) acc[m] = fmaf(S[static_cast<size_t>(r) * C + j0 + jj], vv, acc[m]);
+        for (int u = 0; u < 4; ++u) {
+          const float* vrow = stage + (jj + u) * d + c0;
+          if (cpt == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(vrow);
+            o0[0] = fmaf(pav[u], v.x, o0[0]); o0[1] = fmaf(pav[u], v.y, o0[1]);
+            o0[2] = fmaf(pav[u], v.z, o0[2]); o0[3] = fmaf(pav[u], v.w, o0[3]);
+            o1[0] = fmaf(pbv[u], v.x, o1[0]); o1[1] = fmaf(pbv[u], v.y, o1[1]);
+            o1[2] = fmaf(pbv[u], v.z, o1[2]); o1[3] = fmaf(pbv[u], v.w, o1[3]);
+          } else {
+            const float2 v = *reinterpret_cast<const float2*>(vrow);
+            o0[0] = fmaf(pav[u], v.x, o0[0]); o0[1] = fmaf(pav[u], v.y, o0[1]);
+            o1[0] = fmaf(pbv[u], v.x, o1[0]); o1[1] = fmaf(pbv[u], v.y, o1[1]);
+          }
+        }
       }
     }
   }
 #pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    const int r = rg + G * m;
-    if (r < rows) o_coarse[(static_cast<long long>(bh) * C + i0 + r) * d + e] = acc[m];
+  for (int c = 0; c < 4; ++c) {
+    if (c >= cpt) break;
+    if (r0 < rows) o_coarse[(static_cast<long long>(bh) * C + i0 + r0) * d + c0 + c] = o0[c];
+    if (r0 + 1 < rows) o_coarse[(static_cast<long long>(bh) * C + i0 + r0 + 1) * d + c0 + c] = o1[c];
   }
 }
 
 }  // namespace
 
-// Rows of query cubes per coarse CTA: as many as the smem logits budget
-// allows, at most 16 (the O_c accumulation keeps 16 rows per thread for d=64
-// and 8 for d=128).
+// Rows of query cubes per coarse CTA: 16, or fewer when a [R][C] float32
+// logits block would not fit next to the staging buffers.
 int coarse_rows_per_cta(int C, int d) {
-  int R = kLogitBudgetBytes / (C * 4);
-  const int cap = (d == 128) ? 16 : 16;
-  if (R > cap) R = cap;
-  if (R < 1) R = 1;
+  (void)d;
+  const int Cp = (C + 3) & ~3;
+  int R = 16;
+  while (R > 4 && static_cast<long long>(R) * Cp * 4 > kLogitBudgetBytes) R >>= 1;
   return R;
 }
 
 size_t coarse_smem_bytes(int C, int d, int R) {
-  return (static_cast<size_t>(R) * C + static_cast<size_t>(R) * d +
-          static_cast<size_t>(kKeyChunk) * (d + 1)) * sizeof(float) + 8 * 256 * sizeof(int);
+  const size_t Cp = (static_cast<size_t>(C) + 3) & ~static_cast<size_t>(3);
+  return (R * Cp + static_cast<size_t>(d) * 16 + static_cast<size_t>(kSlice) * kStagePitch) *
+             sizeof(float) + 8 * 256 * sizeof(int);
 }
 
 cudaError_t launch_coarse_select(const Geom& g, const void* qt, const void* kt, const void* vt,

@@ -99,67 +99,121 @@ __device__ __forceinline__ void fail(const Shared& sh, int* status) {
   *sh.abort_flag = 1;
 }
 
+// 2^x with one MUFU operation (ex2.approx, flushes subnormal results to 0;
+// 2^-inf = 0).  The probabilities it feeds are rounded to bf16 afterwards.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
   const __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&p);
 }
 
 // ------------------------------------------------------------------ producer
+// Selection indices of one list, fetched 32 at a time into the lanes of the
+// producer warp (one index per lane) with the next window already in flight,
+// so the slot loads never wait on a global load.
+struct IndexWindow {
+  const int32_t* list;
+  int base, cur, nxt;
+};
+
+__device__ __forceinline__ int fetch_index(const int32_t* list, int i, int topk) {
+  return i < topk ? __ldg(&list[i]) : 0;
+}
+
+__device__ __forceinline__ void window_init(IndexWindow& w, const int32_t* list, int topk,
+                                            int lane) {
+  w.list = list;
+  w.base = 0;
+  w.cur = fetch_index(list, lane, topk);
+  w.nxt = fetch_index(list, 32 + lane, topk);
+}
+
+// Warp-collective: returns list[a] on every lane; a never decreases.
+__device__ __forceinline__ int window_get(IndexWindow& w, int a, int topk, int lane) {
+  while (a >= w.base + 32) {
+    w.base += 32;
+    w.cur = w.nxt;
+    w.nxt = fetch_index(w.list, w.base + 32 + lane, topk);
+  }
+  return __shfl_sync(0xffffffffu, w.cur, a - w.base);
+}
+
+// Run by the whole producer warp; lane 0 issues the barrier and TMA operations.
 template <int D>
 __device__ void producer(const Shared& sh, const Geom& g, const CUtensorMap* tq,
                          const CUtensorMap* tk, const CUtensorMap* tv,
                          const int32_t* __restrict__ counts, const int32_t* __restrict__ sel,
                          int topk, int* status) {
   using Cf = Cfg<D>;
+  const int lane = threadIdx.x & 31;
+  const bool leader = lane == 0;
   const int pairs = (g.C + 1) / 2;
   const int items = g.B * g.H * pairs;
   const int nsteps = (topk + 1) / 2;
   uint32_t ring = 0;
   int t = 0;
+  // lane 0 waits; the verdict is broadcast so the warp leaves together
+  auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+    int ok = 1;
+    if (leader) ok = mbar_wait(bar, parity) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  };
   for (int item = blockIdx.x; item < items; item += gridDim.x, ++t) {
     if (*sh.abort_flag) return;
     const Item it = decode(g, item, pairs);
-    if (__ldg(&counts[it.i0]) != cube_valid(g, it.i0) ||
-        (it.has_b && __ldg(&counts[it.i1]) != cube_valid(g, it.i1)))
+    if (leader && (__ldg(&counts[it.i0]) != cube_valid(g, it.i0) ||
+                   (it.has_b && __ldg(&counts[it.i1]) != cube_valid(g, it.i1))))
       report(status, VSA_ERR_BAD_INDEX);
+    IndexWindow win[2];
+    const int32_t* list0 = sel + (static_cast<long long>(it.bh) * g.C + it.i0) * topk;
+    window_init(win[0], list0, topk, lane);
+    window_init(win[1], it.has_b ? list0 + topk : list0, topk, lane);
     // ---- query tiles of both cubes
     const int qb = t & 1;
-    if (!mbar_wait(&sh.q_empty[qb], ((t >> 1) & 1) ^ 1)) return fail(sh, status);
-    mbar_arrive_expect_tx(&sh.q_full[qb], (it.has_b ? 2 : 1) * Cf::kQBytes);
-    uint8_t* qdst = sh.base + qb * 2 * Cf::kQBytes;
+    if (!wait_all(&sh.q_empty[qb], ((t >> 1) & 1) ^ 1)) return fail(sh, status);
+    if (leader) {
+      mbar_arrive_expect_tx(&sh.q_full[qb], (it.has_b ? 2 : 1) * Cf::kQBytes);
+      uint8_t* qdst = sh.base + qb * 2 * Cf::kQBytes;
 #pragma unroll
-    for (int h = 0; h < Cf::kHalves; ++h) {
-      tma_load_2d(qdst + h * Cf::kQHalf, tq, &sh.q_full[qb], h * 64, it.row0 + it.i0 * 64);
-      if (it.has_b)
-        tma_load_2d(qdst + Cf::kQBytes + h * Cf::kQHalf, tq, &sh.q_full[qb], h * 64,
-                    it.row0 + it.i1 * 64);
+      for (int h = 0; h < Cf::kHalves; ++h) {
+        tma_load_2d(qdst + h * Cf::kQHalf, tq, &sh.q_full[qb], h * 64, it.row0 + it.i0 * 64);
+        if (it.has_b)
+          tma_load_2d(qdst + Cf::kQBytes + h * Cf::kQHalf, tq, &sh.q_full[qb], h * 64,
+                      it.row0 + it.i1 * 64);
+      }
     }
     // ---- key / value slots, in the MMA issuer's order
-    const int32_t* list0 = sel + (static_cast<long long>(it.bh) * g.C + it.i0) * topk;
-    const int32_t* list1 = list0 + topk;
-    int prev0 = -1, prev1 = -1;
+    int prev[2] = {-1, -1};
     auto load = [&](int c, int j, bool is_v) -> bool {
       const int slot = static_cast<int>(ring % Cf::kSlots);
       const uint32_t round = ring / Cf::kSlots;
       ++ring;
-      if (!mbar_wait(&sh.kv_empty[slot], (round & 1u) ^ 1u)) return false;
       const int a = 2 * j;
       const int nk = (a + 1 < topk) ? 2 : 1;
-      mbar_arrive_expect_tx(&sh.kv_full[slot], nk * 64 * D * 2);
-      uint8_t* dst = sh.base + Cf::kRingOff + slot * Cf::kSlotBytes;
-      const int32_t* list = c == 0 ? list0 : list1;
-      int& prev = c == 0 ? prev0 : prev1;
-      for (int r = 0; r < nk; ++r) {
-        int jr = __ldg(&list[a + r]);
-        if (!is_v) {  // validate once per index (on the key load)
-          if (jr < 0 || jr >= g.C || jr <= prev) report(status, VSA_ERR_BAD_INDEX);
-          prev = jr;
-        }
-        jr = jr < 0 ? 0 : (jr >= g.C ? g.C - 1 : jr);
+      int jr[2];
+      jr[0] = window_get(win[c], a, topk, lane);
+      jr[1] = window_get(win[c], a + nk - 1, topk, lane);
+      if (!wait_all(&sh.kv_empty[slot], (round & 1u) ^ 1u)) return false;
+      if (leader) {
+        mbar_arrive_expect_tx(&sh.kv_full[slot], nk * 64 * D * 2);
+        uint8_t* dst = sh.base + Cf::kRingOff + slot * Cf::kSlotBytes;
+        for (int r = 0; r < nk; ++r) {
+          int x = jr[r];
+          if (!is_v) {  // validate once per index (on the key load)
+            if (x < 0 || x >= g.C || x <= prev[c]) report(status, VSA_ERR_BAD_INDEX);
+            prev[c] = x;
+          }
+          x = x < 0 ? 0 : (x >= g.C ? g.C - 1 : x);
 #pragma unroll
-        for (int h = 0; h < Cf::kHalves; ++h)
-          tma_load_2d(dst + h * Cf::kKVHalf + r * (64 * 128), is_v ? tv : tk, &sh.kv_full[slot],
-                      h * 64, it.row0 + jr * 64);
+          for (int h = 0; h < Cf::kHalves; ++h)
+            tma_load_2d(dst + h * Cf::kKVHalf + r * (64 * 128), is_v ? tv : tk,
+                        &sh.kv_full[slot], h * 64, it.row0 + x * 64);
+        }
       }
       return true;
     };
@@ -288,11 +342,13 @@ __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c
     const int ni = cube_valid(g, i);
     const int32_t* list = sel + (static_cast<long long>(it.bh) * g.C + i) * topk;
     float m_ref = -INFINITY, l_part = 0.f;
+    int next_idx = hh < topk ? __ldg(&list[hh]) : -1;  // key cube of this half, step 0
     for (int j = 0; j < nsteps; ++j) {
-      const int a = 2 * j + hh;
+      int jr = next_idx;
+      const int an = 2 * (j + 1) + hh;  // prefetch the next step's index
+      next_idx = (j + 1 < nsteps && an < topk) ? __ldg(&list[an]) : -1;
       int nh = 0;
-      if (a < topk) {
-        int jr = __ldg(&list[a]);
+      if (2 * j + hh < topk) {
         jr = jr < 0 ? 0 : (jr >= g.C ? g.C - 1 : jr);
         nh = cube_valid(g, jr);
       }
@@ -339,8 +395,8 @@ __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c
       uint32_t pk[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const float p0 = exp2f(fmaf(__uint_as_float(sv[2 * e]), sl2, -m_ref));
-        const float p1 = exp2f(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -m_ref));
+        const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * e]), sl2, -m_ref));
+        const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -m_ref));
         sum += p0 + p1;
         pk[e] = pack2_bf16(p0, p1);
       }
@@ -434,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_fwd_kernel(
   const uint32_t tmem = *tmem_slot;
 
   if (warp == kProducerWarp) {
-    if (lane == 0) producer<D>(sh, g, &tq, &tk, &tv, counts, sel, topk, status);
+    producer<D>(sh, g, &tq, &tk, &tv, counts, sel, topk, status);
   } else if (warp == kMmaWarp) {
     if (lane == 0) mma_issuer<D>(sh, g, tmem, topk, status);
   } else if (warp >= kSoftmaxWarp0) {
