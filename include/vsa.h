@@ -55,7 +55,8 @@ enum vsa_status_code {
   VSA_ERR_UNSUPPORTED = 2,  /* cube not 4x4x4, d not in {64, 128}, device not sm_100 */
   VSA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
   VSA_ERR_TIMEOUT = 4,      /* device: a bounded wait ran out (status word) */
-  VSA_ERR_BAD_INDEX = 5     /* device: cube_count or sel_idx entry inconsistent (status word) */
+  VSA_ERR_BAD_INDEX = 5,    /* device: cube_count or sel_idx entry inconsistent (status word) */
+  VSA_ERR_TOO_LARGE = 6     /* problem needs more scratch than vsa_coarse_select_noalloc holds */
 };
 
 typedef struct vsa_shape {
@@ -110,6 +111,32 @@ int vsa_coarse_select(const vsa_shape* shape, const void* q_tiled, const void* k
                       const void* v_tiled, const int32_t* cube_count, int topk,
                       float* o_coarse, int32_t* sel_idx, float* coarse_logits,
                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* vsa_coarse_select for callers that cannot allocate device memory.  The
+ * pages have no counterpart: this is a library convenience.  Some callers own
+ * no device allocator (a plugin inside a host application that manages all
+ * device memory itself) or must not call cudaMalloc while work is in flight
+ * (it may synchronise the device); they cannot provide the workspace that
+ * vsa_coarse_select needs.  This variant takes the same arguments minus the
+ * workspace and computes the same result with the same kernels, using a
+ * fixed 32 MiB device array inside the library as its scratch.
+ *   - Limit: 3*B*H*C*d*4 bytes of pooled q, k, v must fit in 32 MiB, i.e.
+ *     B*H*C*d <= 2,796,202 (e.g. 12 heads x 1440 cubes x d=128 fits; 40 heads
+ *     of the 21x45x80 grid do not).  Larger problems return VSA_ERR_TOO_LARGE
+ *     before any launch; use vsa_coarse_select with a workspace for them.
+ *   - Every GPU context that loads the library holds the 32 MiB from module
+ *     load until the process exits.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls on a device share the one array: calls that overlap on the
+ *     GPU (different streams, no ordering between them) race on it.  Calls
+ *     ordered on one stream are safe.  The array keeps the last call's
+ *     pooled vectors; every call overwrites what it reads.
+ *   - Allocates nothing: no cudaMalloc / cudaFree or allocating library call. */
+int vsa_coarse_select_noalloc(const vsa_shape* shape, const void* q_tiled, const void* k_tiled,
+                              const void* v_tiled, const int32_t* cube_count, int topk,
+                              float* o_coarse, int32_t* sel_idx, float* coarse_logits,
+                              cudaStream_t stream);
 
 /* Fine stage: block-sparse attention over the selected 64x64 blocks (FastWan
  * article, section "一张卡，秒生视频": the fine block-sparse kernel, 64x64

@@ -284,6 +284,7 @@ const char* vsa_strerror(int code) {
     case VSA_ERR_CUDA: return "CUDA runtime error";
     case VSA_ERR_TIMEOUT: return "device wait timed out";
     case VSA_ERR_BAD_INDEX: return "inconsistent cube_count or sel_idx entry";
+    case VSA_ERR_TOO_LARGE: return "problem exceeds the fixed scratch of vsa_coarse_select_noalloc";
     default: return "unknown status";
   }
 }

@@ -29,10 +29,12 @@ VSA_ERR_UNSUPPORTED = 2
 VSA_ERR_CUDA = 3
 VSA_ERR_TIMEOUT = 4
 VSA_ERR_BAD_INDEX = 5
+VSA_ERR_TOO_LARGE = 6
 
 EXPORTED = ("vsa_num_cubes", "vsa_topk_from_ratio", "vsa_workspace_bytes", "vsa_tile_permute",
-            "vsa_coarse_select", "vsa_block_sparse_fwd", "vsa_combine", "vsa_untile",
-            "vsa_get_status", "vsa_debug_wait_timeout", "vsa_strerror")
+            "vsa_coarse_select", "vsa_coarse_select_noalloc", "vsa_block_sparse_fwd",
+            "vsa_combine", "vsa_untile", "vsa_get_status", "vsa_debug_wait_timeout",
+            "vsa_strerror")
 
 
 class VsaShape(ctypes.Structure):
@@ -56,6 +58,7 @@ _sig = {
     "vsa_tile_permute": (ctypes.c_int, [_SP, _P, _P, _P, _P]),
     "vsa_coarse_select": (ctypes.c_int, [_SP, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P, _P,
                                          ctypes.c_size_t, _P]),
+    "vsa_coarse_select_noalloc": (ctypes.c_int, [_SP, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P, _P]),
     "vsa_block_sparse_fwd": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P]),
     "vsa_combine": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P]),
     "vsa_untile": (ctypes.c_int, [_SP, _P, _P, _P]),
@@ -163,6 +166,26 @@ def vsa_coarse_select(shape, q_tiled, k_tiled, v_tiled, cube_count, topk, sel_id
                                   _ptr(coarse_logits), _ptr(workspace),
                                   workspace.numel() * workspace.element_size(), _stream(stream)),
            "vsa_coarse_select")
+
+
+def vsa_coarse_select_noalloc(shape, q_tiled, k_tiled, v_tiled, cube_count, topk, sel_idx,
+                              o_coarse=None, coarse_logits=None, stream=None):
+    """vsa_coarse_select without a workspace, for callers that cannot
+    allocate device memory; its scratch is a fixed 32 MiB array inside the
+    library (see include/vsa.h for the limit and the sharing rules)."""
+    B, H, N, d, C = _dims(shape)
+    for n, t in (("q_tiled", q_tiled), ("k_tiled", k_tiled), ("v_tiled", v_tiled)):
+        _expect(t, torch.bfloat16, (B, H, 64 * C, d), n)
+    _expect(cube_count, torch.int32, (C,), "cube_count")
+    _expect(sel_idx, torch.int32, (B, H, C, topk), "sel_idx")
+    if o_coarse is not None:
+        _expect(o_coarse, torch.float32, (B, H, C, d), "o_coarse")
+    if coarse_logits is not None:
+        _expect(coarse_logits, torch.float32, (B, H, C, C), "coarse_logits")
+    _check(_lib.vsa_coarse_select_noalloc(ctypes.byref(shape), _ptr(q_tiled), _ptr(k_tiled),
+                                          _ptr(v_tiled), _ptr(cube_count), topk, _ptr(o_coarse),
+                                          _ptr(sel_idx), _ptr(coarse_logits), _stream(stream)),
+           "vsa_coarse_select_noalloc")
 
 
 def vsa_block_sparse_fwd(shape, q_tiled, k_tiled, v_tiled, cube_count, sel_idx, topk,
