@@ -232,13 +232,24 @@ __device__ void producer(const Shared& sh, const Geom& g, const CUtensorMap* tq,
 }
 
 // ------------------------------------------------------------------ MMA issuer
+// One thread issues every MMA.  Its own instruction latency must stay far
+// below the 64 cycles an M = 64, N = 128, K = 16 MMA occupies the tensor
+// pipe, so descriptors are built once per operand tile and each k-step only
+// adds a compile-time offset to the start-address field (the 14-bit field
+// holds smem byte address / 16, which cannot carry for a 227 KB window), and
+// every group of MMAs is fully unrolled.
 template <int D>
 __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int topk,
                            int* status) {
   using Cf = Cfg<D>;
+  constexpr int kK = D / 16;  // k-steps of Q K^T
   const int pairs = (g.C + 1) / 2;
   const int items = g.B * g.H * pairs;
   const int nsteps = (topk + 1) / 2;
+  const bool odd = (topk & 1) != 0;  // last step has 64 keys
+  constexpr uint32_t kIdescQK128 = idesc_bf16_f32(64, 128, false, false);
+  constexpr uint32_t kIdescQK64 = idesc_bf16_f32(64, 64, false, false);
+  const uint32_t ring_base = smem_u32(sh.base + Cf::kRingOff);
   uint32_t ring = 0;
   uint32_t p_phase0 = 0u, p_phase1 = 0u;
   int t = 0;
@@ -249,30 +260,31 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
     if (!mbar_wait(&sh.q_full[qb], (t >> 1) & 1)) return fail(sh, status);
     tc_fence_after();
     const uint32_t qa0 = smem_u32(sh.base + qb * 2 * Cf::kQBytes);
-    const uint32_t qa1 = qa0 + Cf::kQBytes;
-    auto next_slot = [&](int& slot) -> bool {
-      slot = static_cast<int>(ring % Cf::kSlots);
+    const uint64_t qdesc0 = sdesc_sw128(qa0, 16, 1024);
+    const uint64_t qdesc1 = sdesc_sw128(qa0 + Cf::kQBytes, 16, 1024);
+    auto next_slot = [&](uint32_t& addr) -> bool {
+      const uint32_t slot = ring % Cf::kSlots;
       const uint32_t round = ring / Cf::kSlots;
       ++ring;
       if (!mbar_wait(&sh.kv_full[slot], round & 1u)) return false;
       tc_fence_after();
+      addr = ring_base + slot * Cf::kSlotBytes;
       return true;
     };
     // S_c = Q_c K^T over one step's keys
     auto qk = [&](int c, int j) -> bool {
-      int slot;
-      if (!next_slot(slot)) return false;
-      const int nk = (2 * j + 1 < topk) ? 2 : 1;
-      const uint32_t idesc = idesc_bf16_f32(64, 64 * nk, false, false);
-      const uint32_t kb = smem_u32(sh.base + Cf::kRingOff + slot * Cf::kSlotBytes);
-      const uint32_t qa = c == 0 ? qa0 : qa1;
+      uint32_t kb;
+      if (!next_slot(kb)) return false;
+      const uint32_t slot = (ring - 1) % Cf::kSlots;
+      const uint64_t a0 = c == 0 ? qdesc0 : qdesc1;
+      const uint64_t b0 = sdesc_sw128(kb, 16, 1024);
+      const uint32_t idesc = (odd && j == nsteps - 1) ? kIdescQK64 : kIdescQK128;
       const uint32_t dS = tmem + (c == 0 ? Cf::kColS0 : Cf::kColS1);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t ao = (kk >> 2) * Cf::kQHalf + (kk & 3) * 32;
-        const uint32_t bo = (kk >> 2) * Cf::kKVHalf + (kk & 3) * 32;
-        umma_ss(dS, sdesc_sw128(qa + ao, 16, 1024), sdesc_sw128(kb + bo, 16, 1024), idesc,
-                kk > 0 ? 1u : 0u);
+      for (int kk = 0; kk < kK; ++kk) {
+        const uint64_t ao = ((kk >> 2) * Cf::kQHalf + (kk & 3) * 32) >> 4;
+        const uint64_t bo = ((kk >> 2) * Cf::kKVHalf + (kk & 3) * 32) >> 4;
+        umma_ss(dS, a0 + ao, b0 + bo, idesc, kk > 0 ? 1u : 0u);
       }
       umma_commit(&sh.kv_empty[slot]);
       umma_commit(&sh.s_full[c]);
@@ -284,15 +296,19 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
       if (!mbar_wait(&sh.p_full[c], ph)) return false;
       ph ^= 1u;
       tc_fence_after();
-      int slot;
-      if (!next_slot(slot)) return false;
-      const int ksteps = ((2 * j + 1 < topk) ? 2 : 1) * 4;  // 16 keys per MMA
-      const uint32_t vb = smem_u32(sh.base + Cf::kRingOff + slot * Cf::kSlotBytes);
+      uint32_t vb;
+      if (!next_slot(vb)) return false;
+      const uint32_t slot = (ring - 1) % Cf::kSlots;
+      const uint64_t v0 = sdesc_sw128(vb, Cf::kKVHalf, 1024);
       const uint32_t dO = tmem + (c == 0 ? Cf::kColO0 : Cf::kColO1);
       const uint32_t aP = tmem + (c == 0 ? Cf::kColS0 : Cf::kColS1);
-      for (int kk = 0; kk < ksteps; ++kk) {
-        umma_ts(dO, aP + kk * 8, sdesc_sw128(vb + kk * 2048, Cf::kKVHalf, 1024), Cf::kIdescPV,
-                (j > 0 || kk > 0) ? 1u : 0u);
+      const uint32_t acc0 = j > 0 ? 1u : 0u;
+      umma_ts(dO, aP, v0, Cf::kIdescPV, acc0);
+#pragma unroll
+      for (int kk = 1; kk < 4; ++kk) umma_ts(dO, aP + kk * 8, v0 + (kk * 2048 >> 4), Cf::kIdescPV, 1u);
+      if (!(odd && j == nsteps - 1)) {
+#pragma unroll
+        for (int kk = 4; kk < 8; ++kk) umma_ts(dO, aP + kk * 8, v0 + (kk * 2048 >> 4), Cf::kIdescPV, 1u);
       }
       umma_commit(&sh.kv_empty[slot]);
       if (j == nsteps - 1) umma_commit(&sh.o_full[c]);
@@ -357,13 +373,18 @@ __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c
       tc_fence_after();
       uint32_t sv[64];
       tmem_ld_16x32bx2_x64(tS, sv);
-      float mx = -INFINITY;
+      if (nh < 64) {  // partial or absent key cube: mask its pad slots
 #pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        const float x = e < nh ? __uint_as_float(sv[e]) : -INFINITY;
-        sv[e] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+        for (int e = 0; e < 64; ++e)
+          if (e >= nh) sv[e] = __float_as_uint(-INFINITY);
       }
+      float mx8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(sv[u]);
+#pragma unroll
+      for (int e = 8; e < 64; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sv[e]));
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       const float mx2 = mx * sl2;
       float alpha = 1.f;
@@ -391,16 +412,17 @@ __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c
         }
       }
       l_part *= alpha;
-      float sum = 0.f;
+      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       uint32_t pk[32];
+      const float neg_m = -m_ref;
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * e]), sl2, -m_ref));
-        const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -m_ref));
-        sum += p0 + p1;
+        const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * e]), sl2, neg_m));
+        const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, neg_m));
+        sum8[e & 7] += p0 + p1;
         pk[e] = pack2_bf16(p0, p1);
       }
-      l_part += sum;
+      l_part += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       tmem_st_16x32bx2_x32(tS, pk);  // P over the first 64 columns of S
       tmem_wait_st();
       tc_fence_before();
