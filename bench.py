@@ -345,7 +345,7 @@ def run_gpu(args, w):
     if rank == 0:
         hbm_bytes = {
             "tile_permute": 3 * w.batch * w.heads * (w.tokens + 64 * w.cubes) * w.head_dim * 2,
-            "untile": w.batch * w.heads * (w.tokens + 64 * w.cubes) * w.head_dim * 2,
+            "untile": w.batch * w.heads * 2 * w.tokens * w.head_dim * 2,  # valid rows in, tokens out
         }
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -374,7 +374,7 @@ def run_gpu(args, w):
 
 # Revision tag of the fine kernel; ncu traffic figures are only reported for
 # the revision they were captured on.
-KERNEL_REV = "fine-v1"
+KERNEL_REV = "fine-v3"
 
 
 def main():
