@@ -153,8 +153,8 @@ def blas_threads():
 
 
 def run_reference(args, w):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    from video_dit_block_vsa_b200 import dist as vdist
+    if vdist.rank_info().rank != 0:  # rank 0 alone times the CPU oracle
         return 0
     x = wl.make_inputs(w)
     per_step_budget = 8.0
@@ -194,15 +194,12 @@ def config_dict(w):
 
 def run_gpu(args, w):
     import torch
-    import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from video_dit_block_vsa_b200 import dist as vdist
+    ri = vdist.rank_info()
+    world, rank, local = ri.world, ri.rank, ri.local_rank
     torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    vdist.init("nccl")
 
     from video_dit_block_vsa_b200 import vsa
 
@@ -254,8 +251,7 @@ def run_gpu(args, w):
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
-    if world > 1:
-        dist.barrier()
+    vdist.barrier(ri)
     torch.cuda.synchronize()
     clocks.start()
     t_start = torch.cuda.Event(enable_timing=True)
@@ -265,21 +261,16 @@ def run_gpu(args, w):
         step(evs[s])
     t_end.record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    vdist.barrier(ri)
     clk = clocks.stop()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = vdist.max_over_ranks(t_start.elapsed_time(t_end), ri, dev)
     status = vsa.vsa_get_status()
     if status != 0:
         raise RuntimeError(f"device status after timed steps: {vsa.vsa_strerror(status)}")
     stage_ms = {name: statistics.mean(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps))
                 for i, name in enumerate(stages)}
     ms_per_step = elapsed_ms / args.steps
-    value = world * step_flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = vdist.job_throughput(step_flops, args.steps, elapsed_ms, world) / 1e12
 
     # ---- end to end through host buffers (pinned), copies inside the timed region
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
@@ -299,8 +290,7 @@ def run_gpu(args, w):
 
     e2e_step()
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    vdist.barrier(ri)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -308,11 +298,7 @@ def run_gpu(args, w):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = vdist.max_over_ranks(e0.elapsed_time(e1), ri, dev)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     if w.gated:
         h2d += hgf.numel() * 4 + hgc.numel() * 4
@@ -355,7 +341,7 @@ def run_gpu(args, w):
             "config": config_dict(w),
             "roofline": roofline,
             "cpu_baseline": cpu,
-            "e2e": {"value": world * step_flops * args.steps / (e2e_ms * 1e-3) / 1e12,
+            "e2e": {"value": vdist.job_throughput(step_flops, args.steps, e2e_ms, world) / 1e12,
                     "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms / args.steps},
             "gpu_launches": launches_per_step * args.steps,
@@ -366,9 +352,7 @@ def run_gpu(args, w):
             "kernel_rev": KERNEL_REV,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    vdist.shutdown(ri)
     return 0
 
 
