@@ -31,19 +31,21 @@ __device__ __forceinline__ long long slot_token(const Geom& g, int c, int s) {
 __global__ void __launch_bounds__(256) tile_permute_kernel(Geom g, const uint4* __restrict__ x,
                                                            uint4* __restrict__ xt,
                                                            int32_t* __restrict__ counts) {
+  // All row indices fit in 32 bits (the host rejects B*H*64*C >= 2^31), so
+  // the per-chunk divisions are 32-bit; only byte offsets are 64-bit.
   const int lg_ch = (g.d == 128) ? 4 : 3;  // 16-byte chunks per row: d/8
-  const long long total = static_cast<long long>(g.B) * g.H * g.rows << lg_ch;
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (long long o = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; o < total;
-       o += stride) {
-    const long long row = o >> lg_ch;
-    const int ch = static_cast<int>(o & ((1 << lg_ch) - 1));
-    const long long bh = row / g.rows;
-    const int r = static_cast<int>(row - bh * g.rows);
-    const long long n = slot_token(g, r >> 6, r & 63);
+  const unsigned rows = static_cast<unsigned>(g.rows);
+  const unsigned total_rows = static_cast<unsigned>(g.B * g.H) * rows;
+  const unsigned rows_per_pass = (gridDim.x * blockDim.x) >> lg_ch;
+  const int ch = threadIdx.x & ((1 << lg_ch) - 1);
+  for (unsigned row = (blockIdx.x * blockDim.x + threadIdx.x) >> lg_ch; row < total_rows;
+       row += rows_per_pass) {
+    const unsigned bh = row / rows;
+    const unsigned r = row - bh * rows;
+    const long long n = slot_token(g, static_cast<int>(r >> 6), static_cast<int>(r & 63));
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (n >= 0) v = __ldg(&x[((bh * g.N + n) << lg_ch) + ch]);
-    xt[o] = v;
+    if (n >= 0) v = __ldg(&x[((static_cast<long long>(bh) * g.N + n) << lg_ch) + ch]);
+    xt[(static_cast<long long>(row) << lg_ch) + ch] = v;
   }
   if (counts != nullptr && blockIdx.x == 0) {
     for (int c = threadIdx.x; c < g.C; c += blockDim.x) counts[c] = cube_valid(g, c);
@@ -53,23 +55,25 @@ __global__ void __launch_bounds__(256) tile_permute_kernel(Geom g, const uint4* 
 __global__ void __launch_bounds__(256) untile_kernel(Geom g, const uint4* __restrict__ xt,
                                                      uint4* __restrict__ x) {
   const int lg_ch = (g.d == 128) ? 4 : 3;
-  const long long total = static_cast<long long>(g.B) * g.H * g.N << lg_ch;
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (long long o = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; o < total;
-       o += stride) {
-    const long long tok = o >> lg_ch;
-    const int ch = static_cast<int>(o & ((1 << lg_ch) - 1));
-    const long long bh = tok / g.N;
-    const long long n = tok - bh * g.N;
-    const int xg = static_cast<int>(n % g.X);
-    const long long ty = n / g.X;
-    const int yg = static_cast<int>(ty % g.Y);
-    const int tg = static_cast<int>(ty / g.Y);
+  const unsigned N = static_cast<unsigned>(g.N);
+  const unsigned total_tok = static_cast<unsigned>(g.B * g.H) * N;
+  const unsigned tok_per_pass = (gridDim.x * blockDim.x) >> lg_ch;
+  const int ch = threadIdx.x & ((1 << lg_ch) - 1);
+  for (unsigned tok = (blockIdx.x * blockDim.x + threadIdx.x) >> lg_ch; tok < total_tok;
+       tok += tok_per_pass) {
+    const unsigned bh = tok / N;
+    const unsigned n = tok - bh * N;
+    const unsigned ty = n / static_cast<unsigned>(g.X);
+    const int xg = static_cast<int>(n - ty * static_cast<unsigned>(g.X));
+    const unsigned tg_u = ty / static_cast<unsigned>(g.Y);
+    const int yg = static_cast<int>(ty - tg_u * static_cast<unsigned>(g.Y));
+    const int tg = static_cast<int>(tg_u);
     const int c = ((tg >> 2) * g.Cy + (yg >> 2)) * g.Cx + (xg >> 2);
     int nt, ny, nx, t0, y0, x0;
     cube_extent(g, c, nt, ny, nx, t0, y0, x0);
     const int s = ((tg - t0) * ny + (yg - y0)) * nx + (xg - x0);
-    x[o] = __ldg(&xt[((bh * g.rows + c * kSlots + s) << lg_ch) + ch]);
+    x[(static_cast<long long>(tok) << lg_ch) + ch] =
+        __ldg(&xt[((static_cast<long long>(bh) * g.rows + c * kSlots + s) << lg_ch) + ch]);
   }
 }
 
@@ -88,14 +92,15 @@ __global__ void __launch_bounds__(256) combine_kernel(Geom g, const uint4* of,
                                                       const float* __restrict__ gc,
                                                       uint4* out) {
   const int lg_ch = (g.d == 128) ? 4 : 3;
-  const long long total = static_cast<long long>(g.B) * g.H * g.rows << lg_ch;
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (long long o = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; o < total;
-       o += stride) {
-    const long long row = o >> lg_ch;
-    const int ch = static_cast<int>(o & ((1 << lg_ch) - 1));
-    const long long bh = row / g.rows;
-    const int r = static_cast<int>(row - bh * g.rows);
+  const unsigned rows = static_cast<unsigned>(g.rows);
+  const unsigned total_rows = static_cast<unsigned>(g.B * g.H) * rows;
+  const unsigned rows_per_pass = (gridDim.x * blockDim.x) >> lg_ch;
+  const int ch = threadIdx.x & ((1 << lg_ch) - 1);
+  for (unsigned row_u = (blockIdx.x * blockDim.x + threadIdx.x) >> lg_ch; row_u < total_rows;
+       row_u += rows_per_pass) {
+    const long long o = (static_cast<long long>(row_u) << lg_ch) + ch;
+    const long long bh = row_u / rows;
+    const int r = static_cast<int>(row_u - static_cast<unsigned>(bh) * rows);
     const int c = r >> 6;
     const long long n = slot_token(g, c, r & 63);
     uint4 res = make_uint4(0u, 0u, 0u, 0u);
