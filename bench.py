@@ -117,29 +117,38 @@ class ClockSampler:
 # ------------------------------------------------------------------ oracle (CPU)
 
 def oracle_sample(w, x, time_budget_s, cubes_cap=None):
-    """Runs the oracle on head 0 of batch 0: the whole coarse stage, then the
-    fine stage for query cubes in order until the time budget or the cap.
+    """Runs the oracle head by head (batch 0, heads 0, 1, ...): for each head the
+    whole coarse stage, then the fine stage for query cubes in order, until the
+    time budget or the cap on query cubes of a head.
     Returns (seconds, effective FLOPs processed, description)."""
     from oracle import vsa_oracle as vo
     t0 = time.perf_counter()
-    one = lambda n: vo.bf16_bits_to_f64(x[n][0:1, 0:1])
-    q_t, counts = vo.tile_permute(one("q"), w.grid)
-    k_t, _ = vo.tile_permute(one("k"), w.grid)
-    v_t, _ = vo.tile_permute(one("v"), w.grid)
-    S, O_c = vo.coarse_attention(vo.pool(q_t, counts), vo.pool(k_t, counts), vo.pool(v_t, counts))
-    sel = vo.topk_select(S, w.topk)
-    C, d = counts.shape[0], w.head_dim
-    flops = 4.0 * d * C * C
-    done = 0
-    while done < C and (cubes_cap is None or done < cubes_cap):
-        vo.block_sparse_attention(q_t, k_t, v_t, counts, sel, query_cubes=[done])
-        flops += 4.0 * d * counts[done] * counts[sel[0, 0, done]].sum()
-        done += 1
-        if time.perf_counter() - t0 > time_budget_s:
+    C, d = w.cubes, w.head_dim
+    flops = 0.0
+    heads_done, last_cubes = 0, 0
+    for h in range(w.heads):
+        one = lambda n: vo.bf16_bits_to_f64(x[n][0:1, h:h + 1])
+        q_t, counts = vo.tile_permute(one("q"), w.grid)
+        k_t, _ = vo.tile_permute(one("k"), w.grid)
+        v_t, _ = vo.tile_permute(one("v"), w.grid)
+        S, O_c = vo.coarse_attention(vo.pool(q_t, counts), vo.pool(k_t, counts), vo.pool(v_t, counts))
+        sel = vo.topk_select(S, w.topk)
+        flops += 4.0 * d * C * C
+        done = 0
+        while done < C and (cubes_cap is None or done < cubes_cap):
+            vo.block_sparse_attention(q_t, k_t, v_t, counts, sel, query_cubes=[done])
+            flops += 4.0 * d * counts[done] * counts[sel[0, 0, done]].sum()
+            done += 1
+            if time.perf_counter() - t0 > time_budget_s:
+                break
+        heads_done, last_cubes = h + 1, done
+        if cubes_cap is not None or time.perf_counter() - t0 > time_budget_s:
             break
     dt = time.perf_counter() - t0
-    desc = (f"head 0 of {w.batch * w.heads}: tile/pool/coarse/top-k over all {C} cubes, "
-            f"fine stage for query cubes 0..{done - 1} ({done} of {C})")
+    full = heads_done - (1 if last_cubes < C else 0)
+    desc = (f"batch 0, heads 0..{heads_done - 1} of {w.batch * w.heads}: tile/pool/coarse/top-k over all "
+            f"{C} cubes of each; fine stage for all query cubes of {full} head(s)"
+            + (f" and cubes 0..{last_cubes - 1} of head {heads_done - 1}" if last_cubes < C else ""))
     return dt, flops, desc
 
 

@@ -149,15 +149,19 @@ __device__ void warp_topk(const float* row, int C, int k, int* hist, int32_t* ou
 // ------------------------------------------------------------------ coarse
 // grid (ceil(C/R), B*H), 256 threads, R <= 16 query cubes per CTA.
 // smem: S [R][Cp] f32 (Cp = C rounded up to 4) | qT [d][16] | staging
-// [32][260] (key slices, then value chunks) | hist [8][256].
+// (key slices [512][33], then value chunks [132][d]) | hist [8][256].
 //
-// Logits: a 16-row x 256-key tile per pass; thread t owns rows 4*(t/64)..+3
-// and keys 4*(t%64)..+3 (16 accumulators), over head-dim slices of 32
-// staged transposed in smem, so each step is two 128-bit smem loads for 16
-// FMAs.  O_c: thread t owns rows 2*(t/32), +1 and d/32 columns.
-constexpr int kTileKeys = 256;
+// Logits: a 16-row x 512-key tile per pass; thread t owns rows 8*(t/128)..+7
+// and keys (t%128) + 128*b, b < 4 (32 accumulators), over head-dim slices of
+// 32 staged row-major at a pitch of 33 floats: the four key loads of a step
+// hit 32 distinct banks per warp, the eight query values are two broadcast
+// 128-bit loads, so a step is six smem wavefronts per warp for 32 FMAs, and
+// the staging stores are conflict-free too.
+// O_c: thread t owns rows 4*(t/64)..+3 and d/64 adjacent columns.
+constexpr int kTileKeys = 512;
 constexpr int kSlice = 32;
-constexpr int kStagePitch = kTileKeys + 4;
+constexpr int kStagePitch = kSlice + 1;
+constexpr int kStageFloats = kTileKeys * kStagePitch;
 
 __global__ void __launch_bounds__(kCoarseThreads) coarse_kernel(
     Geom g, int R, int topk, const float* __restrict__ ws, float* __restrict__ o_coarse,
@@ -167,8 +171,8 @@ __global__ void __launch_bounds__(kCoarseThreads) coarse_kernel(
   const int Cp = (C + 3) & ~3;
   float* S = sm;                                     // [R][Cp]
   float* qT = S + static_cast<size_t>(R) * Cp;       // [d][16]
-  float* stage = qT + static_cast<size_t>(d) * 16;   // [32][kStagePitch]
-  int* hist = reinterpret_cast<int*>(stage + kSlice * kStagePitch);  // [8][256]
+  float* stage = qT + static_cast<size_t>(d) * 16;   // kStageFloats
+  int* hist = reinterpret_cast<int*>(stage + kStageFloats);  // [8][256]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y;
@@ -185,47 +189,51 @@ __global__ void __launch_bounds__(kCoarseThreads) coarse_kernel(
     qT[e] = r < rows ? qbar[static_cast<long long>(i0 + r) * d + col] : 0.f;
   }
   // ---- logits
-  const int rg = tid >> 6, kg = tid & 63;
+  const int rg = tid >> 7, kg = tid & 127;
   for (int j0 = 0; j0 < C; j0 += kTileKeys) {
-    float acc[4][4];
+    float acc[8][4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
       for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
     for (int e0 = 0; e0 < d; e0 += kSlice) {
       __syncthreads();
-      // stage keys j0..j0+255, dims e0..e0+31, transposed: stage[dim][key]
+      // stage keys j0..j0+511, dims e0..e0+31: stage[key][dim], pitch 33
       for (int idx = tid; idx < kTileKeys * (kSlice / 4); idx += kCoarseThreads) {
         const int jj = idx >> 3, q4 = idx & 7;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
         if (j0 + jj < C)
           v = *reinterpret_cast<const float4*>(kbar + static_cast<long long>(j0 + jj) * d + e0 + 4 * q4);
-        stage[(4 * q4 + 0) * kStagePitch + jj] = v.x;
-        stage[(4 * q4 + 1) * kStagePitch + jj] = v.y;
-        stage[(4 * q4 + 2) * kStagePitch + jj] = v.z;
-        stage[(4 * q4 + 3) * kStagePitch + jj] = v.w;
+        float* dst = stage + jj * kStagePitch + 4 * q4;
+        dst[0] = v.x;
+        dst[1] = v.y;
+        dst[2] = v.z;
+        dst[3] = v.w;
       }
       __syncthreads();
-#pragma unroll 8
+      const float* qcol = qT + e0 * 16 + 8 * rg;
+      const float* krow = stage + kg * kStagePitch;
+#pragma unroll 4
       for (int ee = 0; ee < kSlice; ++ee) {
-        const float4 qv = *reinterpret_cast<const float4*>(qT + (e0 + ee) * 16 + 4 * rg);
-        const float4 kv = *reinterpret_cast<const float4*>(stage + ee * kStagePitch + 4 * kg);
-        const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
-        const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
+        const float4 qa = *reinterpret_cast<const float4*>(qcol + ee * 16);
+        const float4 qb = *reinterpret_cast<const float4*>(qcol + ee * 16 + 4);
+        const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+        float kv[4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int b = 0; b < 4; ++b) kv[b] = krow[b * 128 * kStagePitch + ee];
 #pragma unroll
-          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(qa[a], ka[b], acc[a][b]);
+        for (int a = 0; a < 8; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(qv[a], kv[b], acc[a][b]);
       }
     }
-    const int jb = j0 + 4 * kg;
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const int r = 4 * rg + a;
+    for (int a = 0; a < 8; ++a) {
+      const int r = 8 * rg + a;
       if (r >= rows) continue;
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        const int j = jb + b;
+        const int j = j0 + kg + 128 * b;
         if (j < C) {
           const float s = acc[a][b] * scale;
           S[static_cast<size_t>(r) * Cp + j] = s;
@@ -256,11 +264,11 @@ __global__ void __launch_bounds__(kCoarseThreads) coarse_kernel(
     for (int j = lane; j < Cp; j += 32) row[j] = j < C ? row[j] * inv : 0.f;
   }
   if (o_coarse == nullptr) return;
-  // ---- O_c = P vbar: rows 2*(t/32), +1; columns cpt*(t%32) .. +cpt-1
-  const int cpt = d / 32;  // 4 (d=128) or 2 (d=64)
-  const int r0 = 2 * (tid >> 5), c0 = cpt * (tid & 31);
-  float o0[4] = {0.f, 0.f, 0.f, 0.f}, o1[4] = {0.f, 0.f, 0.f, 0.f};
-  const int vchunk = (kSlice * kStagePitch) / d & ~3;  // value rows per staged chunk
+  // ---- O_c = P vbar: rows 4*(t/64)..+3; columns cpt*(t%64) .. +cpt-1
+  const int cpt = d / 64;  // 2 (d=128) or 1 (d=64)
+  const int r0 = 4 * (tid >> 6), c0 = cpt * (tid & 63);
+  float o[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+  const int vchunk = (kStageFloats / d) & ~3;  // value rows per staged chunk
   for (int j0 = 0; j0 < C; j0 += vchunk) {
     __syncthreads();
     const int nk = min(vchunk, C - j0);
@@ -273,35 +281,40 @@ __global__ void __launch_bounds__(kCoarseThreads) coarse_kernel(
     __syncthreads();
     if (r0 < rows) {
       const float* p0 = S + static_cast<size_t>(r0) * Cp + j0;
-      const float* p1 = p0 + Cp;
       for (int jj = 0; jj < nk; jj += 4) {
-        const float4 pa = *reinterpret_cast<const float4*>(p0 + jj);
-        const float4 pb = *reinterpret_cast<const float4*>(p1 + jj);
-        const float pav[4] = {pa.x, pa.y, pa.z, pa.w};
-        const float pbv[4] = {pb.x, pb.y, pb.z, pb.w};
+        float pv[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          const float4 p = *reinterpret_cast<const float4*>(p0 + a * Cp + jj);
+          pv[a][0] = p.x; pv[a][1] = p.y; pv[a][2] = p.z; pv[a][3] = p.w;
+        }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const float* vrow = stage + (jj + u) * d + c0;
-          if (cpt == 4) {
-            const float4 v = *reinterpret_cast<const float4*>(vrow);
-            o0[0] = fmaf(pav[u], v.x, o0[0]); o0[1] = fmaf(pav[u], v.y, o0[1]);
-            o0[2] = fmaf(pav[u], v.z, o0[2]); o0[3] = fmaf(pav[u], v.w, o0[3]);
-            o1[0] = fmaf(pbv[u], v.x, o1[0]); o1[1] = fmaf(pbv[u], v.y, o1[1]);
-            o1[2] = fmaf(pbv[u], v.z, o1[2]); o1[3] = fmaf(pbv[u], v.w, o1[3]);
-          } else {
+          if (cpt == 2) {
             const float2 v = *reinterpret_cast<const float2*>(vrow);
-            o0[0] = fmaf(pav[u], v.x, o0[0]); o0[1] = fmaf(pav[u], v.y, o0[1]);
-            o1[0] = fmaf(pbv[u], v.x, o1[0]); o1[1] = fmaf(pbv[u], v.y, o1[1]);
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+              o[a][0] = fmaf(pv[a][u], v.x, o[a][0]);
+              o[a][1] = fmaf(pv[a][u], v.y, o[a][1]);
+            }
+          } else {
+            const float v = *vrow;
+#pragma unroll
+            for (int a = 0; a < 4; ++a) o[a][0] = fmaf(pv[a][u], v, o[a][0]);
           }
         }
       }
     }
   }
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    if (c >= cpt) break;
-    if (r0 < rows) o_coarse[(static_cast<long long>(bh) * C + i0 + r0) * d + c0 + c] = o0[c];
-    if (r0 + 1 < rows) o_coarse[(static_cast<long long>(bh) * C + i0 + r0 + 1) * d + c0 + c] = o1[c];
+  for (int a = 0; a < 4; ++a) {
+    if (r0 + a >= rows) break;
+    float* dst = o_coarse + (static_cast<long long>(bh) * C + i0 + r0 + a) * d + c0;
+    if (cpt == 2)
+      *reinterpret_cast<float2*>(dst) = make_float2(o[a][0], o[a][1]);
+    else
+      *dst = o[a][0];
   }
 }
 
@@ -319,7 +332,7 @@ int coarse_rows_per_cta(int C, int d) {
 
 size_t coarse_smem_bytes(int C, int d, int R) {
   const size_t Cp = (static_cast<size_t>(C) + 3) & ~static_cast<size_t>(3);
-  return (R * Cp + static_cast<size_t>(d) * 16 + static_cast<size_t>(kSlice) * kStagePitch) *
+  return (R * Cp + static_cast<size_t>(d) * 16 + static_cast<size_t>(kStageFloats)) *
              sizeof(float) + 8 * 256 * sizeof(int);
 }
 
