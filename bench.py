@@ -281,21 +281,19 @@ def run_gpu(args, w):
     ms_per_step = elapsed_ms / args.steps
     value = vdist.job_throughput(step_flops, args.steps, elapsed_ms, world) / 1e12
 
-    # ---- end to end through host buffers (pinned), copies inside the timed region
+    # ---- end to end through the host-buffer entry point (pinned host memory):
+    # every step copies q, k, v (and gates) in and the output out, in chunks of
+    # heads that overlap the copies with the kernels.
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
     hgf = g_f.cpu().pin_memory() if w.gated else None
     hgc = g_c.cpu().pin_memory() if w.gated else None
     hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    chunk = HOST_CHUNK_HEADS
+    hws = torch.empty(vsa.vsa_forward_host_workspace_bytes(shape, w.topk, chunk, w.gated),
+                      dtype=torch.uint8, device=dev)
 
     def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        if w.gated:
-            g_f.copy_(hgf, non_blocking=True)
-            g_c.copy_(hgc, non_blocking=True)
-        step()
-        hout.copy_(out, non_blocking=True)
+        vsa.vsa_forward_host(shape, w.topk, hq, hk, hv, hout, hws, hgf, hgc, chunk)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -308,6 +306,9 @@ def run_gpu(args, w):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = vdist.max_over_ranks(e0.elapsed_time(e1), ri, dev)
+    status = vsa.vsa_get_status()
+    if status != 0:
+        raise RuntimeError(f"device status after end-to-end steps: {vsa.vsa_strerror(status)}")
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     if w.gated:
         h2d += hgf.numel() * 4 + hgc.numel() * 4
@@ -352,7 +353,8 @@ def run_gpu(args, w):
             "cpu_baseline": cpu,
             "e2e": {"value": vdist.job_throughput(step_flops, args.steps, e2e_ms, world) / 1e12,
                     "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms / args.steps},
+                    "ms_per_step": e2e_ms / args.steps, "api": "vsa_forward_host",
+                    "heads_per_chunk": chunk},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
             "stages_ms": stage_ms,
@@ -364,6 +366,9 @@ def run_gpu(args, w):
     vdist.shutdown(ri)
     return 0
 
+
+# (b, h) planes per chunk of the host-buffer path in the end-to-end leg.
+HOST_CHUNK_HEADS = 8
 
 # Revision tag of the fine kernel; ncu traffic figures are only reported for
 # the revision they were captured on.

@@ -173,6 +173,37 @@ int vsa_combine(const vsa_shape* shape, const void* o_fine_tiled, const float* o
  * pad rows are dropped. */
 int vsa_untile(const vsa_shape* shape, const void* x_tiled, void* x, cudaStream_t stream);
 
+/* Bytes of device workspace vsa_forward_host needs: two chunk buffers, each
+ * holding heads_per_chunk (b, h) planes of the inputs, their tiled copies,
+ * the fine and final outputs and the coarse-stage scratch.  heads_per_chunk
+ * 0 means 8; gated is 0 or 1.  Returns 0 for an invalid shape or k. */
+size_t vsa_forward_host_workspace_bytes(const vsa_shape* shape, int topk, int heads_per_chunk,
+                                        int gated);
+
+/* The whole forward path (tile, coarse stage, fine stage, gated combine,
+ * untile) from HOST buffers, for callers whose tensors live in host memory.
+ * The pages give no such call; it composes the calls above.
+ *   q, k, v   bf16 [B, H, N, d] in token order, HOST memory (read)
+ *   g_fine, g_coarse float32 [B, H, N] HOST memory, or both NULL (ungated)
+ *   out       bf16 [B, H, N, d] HOST memory (written)
+ *   workspace DEVICE memory, 256-byte aligned, of at least
+ *             vsa_forward_host_workspace_bytes(shape, topk, heads_per_chunk, gated)
+ * The B*H planes are processed in chunks of heads_per_chunk (0: 8): while one
+ * chunk computes on `stream`, the library copies the next chunk in and the
+ * previous chunk's output out on two copy streams of its own (created once
+ * per device), so both PCIe directions overlap the kernels.  Host buffers
+ * should be page-locked (cudaHostAlloc / cudaHostRegister); pageable memory
+ * works but its copies do not overlap.  The call returns once everything is
+ * enqueued: `out` is complete when `stream` is (for example after
+ * cudaStreamSynchronize(stream) or vsa_get_status(stream)), and earlier work
+ * on `stream` finishes before the workspace is touched.  Argument errors are
+ * reported before any copy; a failure after some chunks were enqueued
+ * returns its code with those chunks still in flight. */
+int vsa_forward_host(const vsa_shape* shape, int topk, const void* q, const void* k,
+                     const void* v, const float* g_fine, const float* g_coarse, void* out,
+                     void* workspace, size_t workspace_bytes, int heads_per_chunk,
+                     cudaStream_t stream);
+
 /* Synchronises `stream`, then returns and clears the status word of the
  * current device: VSA_OK, VSA_ERR_TIMEOUT or VSA_ERR_BAD_INDEX recorded by a
  * kernel since the last call, or VSA_ERR_CUDA if the synchronisation failed. */

@@ -95,3 +95,40 @@ def test_strerror(vsa):
     assert vsa.vsa_strerror(0) == "ok"
     assert "timed out" in vsa.vsa_strerror(vsa.VSA_ERR_TIMEOUT)
     assert vsa.vsa_strerror(99) == "unknown status"
+
+
+def test_forward_host_workspace_and_argument_checks(vsa):
+    lib = vsa._lib
+    s = vsa.make_shape(1, 40, 128, (21, 45, 80))
+    C, N, d = 1440, 21 * 45 * 80, 128
+    per_chunk_ungated = (3 * 8 * N * d * 2 + 4 * 8 * 64 * C * d * 2 + 8 * N * d * 2
+                         + 8 * C * 180 * 4 + 3 * 8 * C * d * 4 + C * 4)
+    got = vsa.vsa_forward_host_workspace_bytes(s, 180, 8, gated=False)
+    assert per_chunk_ungated * 2 <= got <= per_chunk_ungated * 2 + 2 * 16 * 256
+    gated = vsa.vsa_forward_host_workspace_bytes(s, 180, 8, gated=True)
+    assert gated - got >= 2 * (2 * 8 * N * 4 + 8 * C * d * 4)
+    assert vsa.vsa_forward_host_workspace_bytes(s, 180, 0) == got  # 0 means 8 planes per chunk
+    assert vsa.vsa_forward_host_workspace_bytes(s, 0, 8) == 0
+    assert vsa.vsa_forward_host_workspace_bytes(s, 180, -1) == 0
+    # a chunk never exceeds B*H planes
+    small = vsa.make_shape(1, 2, 64, (4, 8, 8))
+    assert (vsa.vsa_forward_host_workspace_bytes(small, 2, 8)
+            == vsa.vsa_forward_host_workspace_bytes(small, 2, 2))
+
+    p = ctypes.c_void_p(0x1000)
+    ws = ctypes.c_void_p(0x100000)
+    big = ctypes.c_size_t(1 << 40)
+    call = lambda *a: lib.vsa_forward_host(ctypes.byref(small), *a)
+    ok_args = [2, p, p, p, None, None, p, ws, big, 0, None]
+    a = list(ok_args); a[1] = None                       # q missing
+    assert call(*a) == vsa.VSA_ERR_INVALID_ARG
+    a = list(ok_args); a[4] = p                          # one gate without the other
+    assert call(*a) == vsa.VSA_ERR_INVALID_ARG
+    a = list(ok_args); a[7] = ctypes.c_void_p(0x100010)  # workspace not 256-byte aligned
+    assert call(*a) == vsa.VSA_ERR_INVALID_ARG
+    a = list(ok_args); a[8] = ctypes.c_size_t(1024)      # workspace too small
+    assert call(*a) == vsa.VSA_ERR_INVALID_ARG
+    a = list(ok_args); a[0] = 5                          # k > C
+    assert call(*a) == vsa.VSA_ERR_INVALID_ARG
+    a = list(ok_args); a[9] = -2                         # negative chunk
+    assert call(*a) == vsa.VSA_ERR_INVALID_ARG

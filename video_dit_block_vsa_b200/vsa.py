@@ -33,8 +33,8 @@ VSA_ERR_TOO_LARGE = 6
 
 EXPORTED = ("vsa_num_cubes", "vsa_topk_from_ratio", "vsa_workspace_bytes", "vsa_tile_permute",
             "vsa_coarse_select", "vsa_coarse_select_noalloc", "vsa_block_sparse_fwd",
-            "vsa_combine", "vsa_untile", "vsa_get_status", "vsa_debug_wait_timeout",
-            "vsa_strerror")
+            "vsa_combine", "vsa_untile", "vsa_forward_host_workspace_bytes", "vsa_forward_host",
+            "vsa_get_status", "vsa_debug_wait_timeout", "vsa_strerror")
 
 
 class VsaShape(ctypes.Structure):
@@ -62,6 +62,9 @@ _sig = {
     "vsa_block_sparse_fwd": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P]),
     "vsa_combine": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P]),
     "vsa_untile": (ctypes.c_int, [_SP, _P, _P, _P]),
+    "vsa_forward_host_workspace_bytes": (ctypes.c_size_t, [_SP, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+    "vsa_forward_host": (ctypes.c_int, [_SP, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
+                                        ctypes.c_int, _P]),
     "vsa_get_status": (ctypes.c_int, [_P]),
     "vsa_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
     "vsa_strerror": (ctypes.c_char_p, [ctypes.c_int]),
@@ -224,6 +227,42 @@ def vsa_untile(shape, x_tiled, x, stream=None):
     _expect(x, torch.bfloat16, (B, H, N, d), "x")
     _check(_lib.vsa_untile(ctypes.byref(shape), _ptr(x_tiled), _ptr(x), _stream(stream)),
            "vsa_untile")
+
+
+def _expect_host(t, dtype, shape, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.is_cuda:
+        raise ValueError(f"{name}: expected a host (CPU) tensor")
+
+
+def vsa_forward_host_workspace_bytes(shape, topk, heads_per_chunk=0, gated=False) -> int:
+    return int(_lib.vsa_forward_host_workspace_bytes(ctypes.byref(shape), topk, heads_per_chunk,
+                                                     1 if gated else 0))
+
+
+def vsa_forward_host(shape, topk, q, k, v, out, workspace, g_fine=None, g_coarse=None,
+                     heads_per_chunk=0, stream=None):
+    """The whole path from host tensors (pinned for overlap): q, k, v, out bf16
+    [B, H, N, d] and optional gates float32 [B, H, N] on the CPU; workspace is a
+    device uint8 tensor of vsa_forward_host_workspace_bytes.  Asynchronous on
+    ``stream``; ``out`` is complete when the stream is."""
+    B, H, N, d, C = _dims(shape)
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        _expect_host(t, torch.bfloat16, (B, H, N, d), n)
+    if (g_fine is None) != (g_coarse is None):
+        raise ValueError("give both gates or neither")
+    if g_fine is not None:
+        _expect_host(g_fine, torch.float32, (B, H, N), "g_fine")
+        _expect_host(g_coarse, torch.float32, (B, H, N), "g_coarse")
+    if not workspace.is_cuda:
+        raise ValueError("workspace: expected a CUDA tensor")
+    _check(_lib.vsa_forward_host(ctypes.byref(shape), topk, _ptr(q), _ptr(k), _ptr(v), _ptr(g_fine),
+                                 _ptr(g_coarse), _ptr(out), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), heads_per_chunk,
+                                 _stream(stream)), "vsa_forward_host")
 
 
 def vsa_get_status(stream=None) -> int:
