@@ -117,39 +117,65 @@ class ClockSampler:
 # ------------------------------------------------------------------ oracle (CPU)
 
 def oracle_sample(w, x, time_budget_s, cubes_cap=None):
-    """Runs the oracle head by head (batch 0, heads 0, 1, ...): for each head the
-    whole coarse stage, then the fine stage for query cubes in order, until the
-    time budget or the cap on query cubes of a head.
-    Returns (seconds, effective FLOPs processed, description)."""
+    """Runs the oracle head by head (batch 0, heads 0, 1, ...) until the time
+    budget: a head that fits runs the whole path (tile q, k, v; pool, coarse
+    attention, top-k; fine attention over every query cube; combine; untile),
+    the head that meets the budget runs its fine stage cube by cube until it
+    runs out.  ``cubes_cap`` limits the first head to that many query cubes.
+    Returns (seconds, effective FLOPs processed, description, per-stage
+    seconds summed over whole heads, whole heads)."""
     from oracle import vsa_oracle as vo
     t0 = time.perf_counter()
     C, d = w.cubes, w.head_dim
     flops = 0.0
-    heads_done, last_cubes = 0, 0
+    stages = dict(tile_permute=0.0, coarse_select=0.0, block_sparse_fwd=0.0, combine=0.0, untile=0.0)
+    full_heads, partial = 0, None
+
+    def clock(name, fn, *a, **kw):
+        s0 = time.perf_counter()
+        r = fn(*a, **kw)
+        stages_head[name] += time.perf_counter() - s0
+        return r
+
     for h in range(w.heads):
+        stages_head = dict.fromkeys(stages, 0.0)
         one = lambda n: vo.bf16_bits_to_f64(x[n][0:1, h:h + 1])
-        q_t, counts = vo.tile_permute(one("q"), w.grid)
-        k_t, _ = vo.tile_permute(one("k"), w.grid)
-        v_t, _ = vo.tile_permute(one("v"), w.grid)
+        q_t, counts = clock("tile_permute", vo.tile_permute, one("q"), w.grid)
+        k_t, _ = clock("tile_permute", vo.tile_permute, one("k"), w.grid)
+        v_t, _ = clock("tile_permute", vo.tile_permute, one("v"), w.grid)
+        s0 = time.perf_counter()
         S, O_c = vo.coarse_attention(vo.pool(q_t, counts), vo.pool(k_t, counts), vo.pool(v_t, counts))
         sel = vo.topk_select(S, w.topk)
+        stages_head["coarse_select"] += time.perf_counter() - s0
         flops += 4.0 * d * C * C
+        O_f = np.zeros_like(q_t)
         done = 0
         while done < C and (cubes_cap is None or done < cubes_cap):
-            vo.block_sparse_attention(q_t, k_t, v_t, counts, sel, query_cubes=[done])
+            s0 = time.perf_counter()
+            o, _ = vo.block_sparse_attention(q_t, k_t, v_t, counts, sel, query_cubes=[done])
+            stages_head["block_sparse_fwd"] += time.perf_counter() - s0
+            O_f[:, :, 64 * done:64 * done + 64] = o[:, :, 64 * done:64 * done + 64]
             flops += 4.0 * d * counts[done] * counts[sel[0, 0, done]].sum()
             done += 1
             if time.perf_counter() - t0 > time_budget_s:
                 break
-        heads_done, last_cubes = h + 1, done
-        if cubes_cap is not None or time.perf_counter() - t0 > time_budget_s:
+        if done < C:
+            partial = (h, done)
+            break
+        gf = x["g_f"][0:1, h:h + 1].astype(np.float64) if w.gated else None
+        gc = x["g_c"][0:1, h:h + 1].astype(np.float64) if w.gated else None
+        out_t = clock("combine", vo.combine, O_f, O_c, counts, w.grid, gf, gc)
+        clock("untile", vo.untile, out_t, w.grid)
+        for k_ in stages:
+            stages[k_] += stages_head[k_]
+        full_heads += 1
+        if time.perf_counter() - t0 > time_budget_s:
             break
     dt = time.perf_counter() - t0
-    full = heads_done - (1 if last_cubes < C else 0)
-    desc = (f"batch 0, heads 0..{heads_done - 1} of {w.batch * w.heads}: tile/pool/coarse/top-k over all "
-            f"{C} cubes of each; fine stage for all query cubes of {full} head(s)"
-            + (f" and cubes 0..{last_cubes - 1} of head {heads_done - 1}" if last_cubes < C else ""))
-    return dt, flops, desc
+    desc = (f"batch 0: the whole path for {full_heads} of {w.batch * w.heads} head(s)"
+            + (f", plus tile/coarse/top-k and query cubes 0..{partial[1] - 1} of head {partial[0]}"
+               if partial else ""))
+    return dt, flops, desc, stages, full_heads
 
 
 def blas_threads():
@@ -172,7 +198,7 @@ def run_reference(args, w):
     tot_t = tot_f = 0.0
     desc = ""
     for _ in range(args.steps):
-        dt, fl, desc = oracle_sample(w, x, per_step_budget)
+        dt, fl, desc, _, _ = oracle_sample(w, x, per_step_budget)
         tot_t += dt
         tot_f += fl
     value = tot_f / tot_t / 1e12
@@ -334,9 +360,13 @@ def run_gpu(args, w):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, fl, desc = oracle_sample(w, x, args.cpu_seconds)
+        dt, fl, desc, st, nh = oracle_sample(w, x, args.cpu_seconds)
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
                "kind": "oracle", "sample": desc + f", {dt:.1f} s"}
+        if nh:
+            per_head = {k_: v_ / nh for k_, v_ in st.items()}
+            cpu["stages_s_per_head"] = per_head
+            cpu["s_per_call_extrapolated"] = sum(per_head.values()) * w.batch * w.heads
 
     if rank == 0:
         hbm_bytes = {

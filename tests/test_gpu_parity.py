@@ -77,6 +77,8 @@ COARSE = [  # (B, H, d, grid, k)
     (1, 2, 128, (21, 30, 52), 62),
     (1, 1, 128, (21, 45, 80), 180),
     (1, 1, 64, (16, 32, 32), 256),
+    (1, 1, 64, (48, 48, 48), 200),   # C = 1728: rows longer than the register-cached part
+    (1, 1, 64, (36, 64, 64), 300),   # C = 2304: 8 query cubes per coarse CTA
 ]
 
 
@@ -115,9 +117,10 @@ def test_coarse_select(vsa, B, H, d, grid, k):
     assert vsa.vsa_get_status() == 0
 
 
-def test_topk_ties_go_to_lower_index(vsa):
+@pytest.mark.parametrize("grid,k", [((8, 8, 8), 3), ((48, 48, 48), 1700)])
+def test_topk_ties_go_to_lower_index(vsa, grid, k):
     # identical k vectors in every cube -> all coarse logits of a row tie
-    B, H, d, grid, k = 1, 1, 64, (8, 8, 8), 3
+    B, H, d = 1, 1, 64
     N = math.prod(grid)
     shape = vsa.make_shape(B, H, d, grid)
     C = vsa.vsa_num_cubes(shape)

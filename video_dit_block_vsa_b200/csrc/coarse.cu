@@ -9,9 +9,10 @@
 //      sel[i]    = top-k of S_c[i, :], ties to the lower index, ascending
 //      O_c[i]    = softmax(S_c[i, :]) vbar
 //    The per-row top-k is a warp-level MSB-first radix select on the
-//    order-preserving integer image of the float logits, followed by one
-//    ballot-compaction pass in index order (so the output is ascending and
-//    equal logits are taken lowest index first).
+//    order-preserving integer image of the float logits (kept in registers
+//    for rows of up to 1536 cubes), followed by one ballot-compaction pass in
+//    index order (so the output is ascending and equal logits are taken
+//    lowest index first).
 #include <cmath>
 
 #include "common.cuh"
@@ -77,17 +78,34 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Keys of a row cached in registers per lane (rows of up to 32 * kTopkRegs
+// cubes never re-read shared memory during the selection).
+constexpr int kTopkRegs = 48;
+
 // Writes the indices of the k largest of row[0..C) (ties: lower index first)
 // in ascending order to out[0..k).  Executed by one full warp; hist is a
-// warp-private 256-entry smem array.
+// warp-private 256-entry smem array.  Most-significant-digit-first radix
+// select over the order-preserving integer image of the floats, 8 bits per
+// pass, then one ballot-compaction pass in index order.
 __device__ void warp_topk(const float* row, int C, int k, int* hist, int32_t* out) {
   const int lane = threadIdx.x & 31;
+  uint32_t kc[kTopkRegs];
+#pragma unroll
+  for (int u = 0; u < kTopkRegs; ++u) {
+    const int j = lane + 32 * u;
+    kc[u] = j < C ? order_key(row[j]) : 0u;
+  }
   uint32_t prefix = 0u, mask = 0u;
   int remaining = k;  // rank of the wanted key among the keys matching the prefix
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int b = lane; b < 256; b += 32) hist[b] = 0;
     __syncwarp();
-    for (int j = lane; j < C; j += 32) {
+#pragma unroll
+    for (int u = 0; u < kTopkRegs; ++u) {
+      const int j = lane + 32 * u;
+      if (j < C && (kc[u] & mask) == prefix) atomicAdd(&hist[(kc[u] >> shift) & 255u], 1);
+    }
+    for (int j = lane + 32 * kTopkRegs; j < C; j += 32) {
       const uint32_t key = order_key(row[j]);
       if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
     }
@@ -132,7 +150,19 @@ __device__ void warp_topk(const float* row, int C, int k, int* hist, int32_t* ou
   // `remaining` keys equal to it, in index order.
   const unsigned lt = (1u << lane) - 1u;
   int pos = 0, eq_seen = 0;
-  for (int j0 = 0; j0 < C; j0 += 32) {
+#pragma unroll
+  for (int u = 0; u < kTopkRegs; ++u) {
+    const int j = lane + 32 * u;
+    const bool gt = j < C && kc[u] > prefix;
+    const bool eq = j < C && kc[u] == prefix;
+    const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && eq_seen + __popc(eqm & lt) < remaining);
+    const unsigned tm = __ballot_sync(0xffffffffu, take);
+    if (take) out[pos + __popc(tm & lt)] = j;
+    pos += __popc(tm);
+    eq_seen += __popc(eqm);
+  }
+  for (int j0 = 32 * kTopkRegs; j0 < C; j0 += 32) {
     const int j = j0 + lane;
     const uint32_t key = j < C ? order_key(row[j]) : 0u;
     const bool gt = j < C && key > prefix;
@@ -250,9 +280,11 @@ __global__ void __launch_bounds__(kCoarseThreads) coarse_kernel(
     warp_topk(row, C, topk, hist + warp * 256,
               sel + (static_cast<long long>(bh) * C + i0 + r) * topk);
     float mx = -INFINITY;
+#pragma unroll 8
     for (int j = lane; j < C; j += 32) mx = fmaxf(mx, row[j]);
     for (int off = 16; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     float z = 0.f;
+#pragma unroll 8
     for (int j = lane; j < C; j += 32) {
       const float p = expf(row[j] - mx);
       row[j] = p;
@@ -261,6 +293,7 @@ __global__ void __launch_bounds__(kCoarseThreads) coarse_kernel(
     for (int off = 16; off; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
     const float inv = 1.0f / z;
     __syncwarp();
+#pragma unroll 8
     for (int j = lane; j < Cp; j += 32) row[j] = j < C ? row[j] * inv : 0.f;
   }
   if (o_coarse == nullptr) return;
