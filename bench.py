@@ -352,11 +352,22 @@ def run_gpu(args, w):
             traffic = tj.get("bytes_per_launch")
     except (OSError, ValueError):
         pass
+    # The fine kernel's other roofline: every selected K/V tile and every Q tile
+    # is moved from L2 into shared memory by TMA, and one SM's TMA path sustains
+    # TMA_INGEST_B_PER_CLK with this kernel's box shape.
+    kv_bytes = float(w.batch * w.heads * w.cubes) * (w.topk * 2 + 1) * 64 * w.head_dim * 2
+    sm_hz = 1e6 * ((clk or {}).get("sm_mhz") or 1965.0)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    feed_peak = TMA_INGEST_B_PER_CLK * sms * sm_hz / 1e12
+    feed = {"path": "L2 -> shared memory (TMA)", "bytes": kv_bytes,
+            "achieved": kv_bytes / (fine_ms * 1e-3) / 1e12, "peak": feed_peak, "unit": "TB/s",
+            "frac": kv_bytes / (fine_ms * 1e-3) / 1e12 / feed_peak,
+            "peak_kind": f"{TMA_INGEST_B_PER_CLK} B/clk per SM (measured) x {sms} SMs x {sm_hz / 1e6:.0f} MHz"}
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_sustained"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"], "traffic": traffic,
                 "kernel": "vsa_block_sparse_fwd", "peak_kind": f"bf16 sustained ({peaks['source']})",
                 "peak_burst": peaks["bf16"], "frac_of_burst": achieved / peaks["bf16"],
-                "issued_tflops": fine_issued / (fine_ms * 1e-3) / 1e12}
+                "issued_tflops": fine_issued / (fine_ms * 1e-3) / 1e12, "feed": feed}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -397,8 +408,13 @@ def run_gpu(args, w):
     return 0
 
 
+# Sustained TMA ingest of one SM (bytes per SM clock) for random 64-row x 128-byte
+# swizzled boxes from L2, measured on B200 with 2 to 6 ring slots and 37 to 148
+# SMs loading at once (the figure did not move with either).
+TMA_INGEST_B_PER_CLK = 42.2
+
 # (b, h) planes per chunk of the host-buffer path in the end-to-end leg.
-HOST_CHUNK_HEADS = 8
+HOST_CHUNK_HEADS = 2
 
 # Revision tag of the fine kernel; ncu traffic figures are only reported for
 # the revision they were captured on.

@@ -176,7 +176,7 @@ int vsa_untile(const vsa_shape* shape, const void* x_tiled, void* x, cudaStream_
 /* Bytes of device workspace vsa_forward_host needs: two chunk buffers, each
  * holding heads_per_chunk (b, h) planes of the inputs, their tiled copies,
  * the fine and final outputs and the coarse-stage scratch.  heads_per_chunk
- * 0 means 8; gated is 0 or 1.  Returns 0 for an invalid shape or k. */
+ * 0 means 2; gated is 0 or 1.  Returns 0 for an invalid shape or k. */
 size_t vsa_forward_host_workspace_bytes(const vsa_shape* shape, int topk, int heads_per_chunk,
                                         int gated);
 
@@ -188,7 +188,7 @@ size_t vsa_forward_host_workspace_bytes(const vsa_shape* shape, int topk, int he
  *   out       bf16 [B, H, N, d] HOST memory (written)
  *   workspace DEVICE memory, 256-byte aligned, of at least
  *             vsa_forward_host_workspace_bytes(shape, topk, heads_per_chunk, gated)
- * The B*H planes are processed in chunks of heads_per_chunk (0: 8): while one
+ * The B*H planes are processed in chunks of heads_per_chunk (0: 2): while one
  * chunk computes on `stream`, the library copies the next chunk in and the
  * previous chunk's output out on two copy streams of its own (created once
  * per device), so both PCIe directions overlap the kernels.  Host buffers

@@ -59,7 +59,7 @@ def host_path(vsa, w, x, shape, heads_per_chunk, repeats=1):
 CASES = [
     (wl.WORKLOADS["tiny_k2"], 1),                # 2 planes, one per chunk
     (wl.WORKLOADS["wan1.3b_ft_16x28x52"], 5),    # gated, 12 planes: chunks 5, 5, 2
-    (wl.WORKLOADS["scaling_16x32x32"], 0),       # ungated, default chunk of 8: 8, 4
+    (wl.WORKLOADS["scaling_16x32x32"], 0),       # ungated, default chunk of 2: six chunks
     (wl.Workload("b2_ragged", 2, 3, 64, (5, 7, 9), 3, 11, 0.5, True), 4),  # chunk crosses b
     (wl.Workload("b3_one_chunk", 3, 1, 128, (6, 6, 10), 4, 12, 0.5, False), 16),
 ]

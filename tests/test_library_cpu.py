@@ -107,7 +107,9 @@ def test_forward_host_workspace_and_argument_checks(vsa):
     assert per_chunk_ungated * 2 <= got <= per_chunk_ungated * 2 + 2 * 16 * 256
     gated = vsa.vsa_forward_host_workspace_bytes(s, 180, 8, gated=True)
     assert gated - got >= 2 * (2 * 8 * N * 4 + 8 * C * d * 4)
-    assert vsa.vsa_forward_host_workspace_bytes(s, 180, 0) == got  # 0 means 8 planes per chunk
+    # 0 means 2 planes per chunk
+    assert vsa.vsa_forward_host_workspace_bytes(s, 180, 0) == vsa.vsa_forward_host_workspace_bytes(s, 180, 2)
+    assert vsa.vsa_forward_host_workspace_bytes(s, 180, 2) < got
     assert vsa.vsa_forward_host_workspace_bytes(s, 0, 8) == 0
     assert vsa.vsa_forward_host_workspace_bytes(s, 180, -1) == 0
     # a chunk never exceeds B*H planes

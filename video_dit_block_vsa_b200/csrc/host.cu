@@ -82,7 +82,7 @@ bool shape_ok(const vsa_shape* s, int topk, int* C, long long* N) {
 
 int chunk_heads(const vsa_shape* s, int heads_per_chunk) {
   const int bh = s->batch * s->heads;
-  int hc = heads_per_chunk > 0 ? heads_per_chunk : 8;
+  int hc = heads_per_chunk > 0 ? heads_per_chunk : 2;
   return hc < bh ? hc : bh;
 }
 
