@@ -354,15 +354,14 @@ def run_gpu(args, w):
         pass
     # The fine kernel's other roofline: every selected K/V tile and every Q tile
     # is moved from L2 into shared memory by TMA, and one SM's TMA path sustains
-    # TMA_INGEST_B_PER_CLK with this kernel's box shape.
+    # TMA_INGEST_GBS_PER_SM with this kernel's box shape.
     kv_bytes = float(w.batch * w.heads * w.cubes) * (w.topk * 2 + 1) * 64 * w.head_dim * 2
-    sm_hz = 1e6 * ((clk or {}).get("sm_mhz") or 1965.0)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    feed_peak = TMA_INGEST_B_PER_CLK * sms * sm_hz / 1e12
+    feed_peak = TMA_INGEST_GBS_PER_SM * sms / 1e3
     feed = {"path": "L2 -> shared memory (TMA)", "bytes": kv_bytes,
             "achieved": kv_bytes / (fine_ms * 1e-3) / 1e12, "peak": feed_peak, "unit": "TB/s",
             "frac": kv_bytes / (fine_ms * 1e-3) / 1e12 / feed_peak,
-            "peak_kind": f"{TMA_INGEST_B_PER_CLK} B/clk per SM (measured) x {sms} SMs x {sm_hz / 1e6:.0f} MHz"}
+            "peak_kind": f"{TMA_INGEST_GBS_PER_SM} GB/s per SM (measured) x {sms} SMs"}
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_sustained"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"], "traffic": traffic,
                 "kernel": "vsa_block_sparse_fwd", "peak_kind": f"bf16 sustained ({peaks['source']})",
@@ -408,17 +407,17 @@ def run_gpu(args, w):
     return 0
 
 
-# Sustained TMA ingest of one SM (bytes per SM clock) for random 64-row x 128-byte
-# swizzled boxes from L2, measured on B200 with 2 to 6 ring slots and 37 to 148
-# SMs loading at once (the figure did not move with either).
-TMA_INGEST_B_PER_CLK = 42.2
+# Sustained TMA ingest of one SM for random 64-row x 128-byte swizzled boxes from
+# L2, measured on B200 (the best of two probe layouts; the figure did not move
+# with 2 to 6 ring slots or with 37 to 148 SMs loading at once).
+TMA_INGEST_GBS_PER_SM = 99.3
 
 # (b, h) planes per chunk of the host-buffer path in the end-to-end leg.
 HOST_CHUNK_HEADS = 2
 
 # Revision tag of the fine kernel; ncu traffic figures are only reported for
 # the revision they were captured on.
-KERNEL_REV = "fine-v3"
+KERNEL_REV = "fine-v3.2"
 
 
 def main():

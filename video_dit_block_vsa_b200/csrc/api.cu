@@ -111,6 +111,8 @@ int make_geom(const vsa_shape* s, Geom* g) {
   g->C = static_cast<int>(C);
   g->N = static_cast<long long>(g->T) * g->Y * g->X;
   g->rows = C * kSlots;
+  g->inv_cx = ((1ull << 32) + g->Cx - 1) / g->Cx;
+  g->inv_cy = ((1ull << 32) + g->Cy - 1) / g->Cy;
   const long long all_rows = static_cast<long long>(g->B) * g->H * g->rows;
   if (all_rows >= (1ll << 31) || static_cast<long long>(g->B) * g->H >= 65536)
     return VSA_ERR_UNSUPPORTED;

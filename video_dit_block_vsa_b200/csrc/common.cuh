@@ -22,15 +22,25 @@ struct Geom {
   int C;             // cubes
   long long N;       // tokens
   long long rows;    // 64*C tiled rows per (b, h)
+  uint64_t inv_cx;   // ceil(2^32 / Cx): for n, Cx < 2^16, n / Cx == (n * inv_cx) >> 32
+  uint64_t inv_cy;   // ceil(2^32 / Cy)
 };
+
+// Division by a runtime divisor below 2^16 for dividends below 2^16, with the
+// precomputed reciprocal inv = ceil(2^32 / d): n * inv / 2^32 = n / d + n e / (d 2^32)
+// with 0 <= e < d, and the second term stays below 1/d when n e < 2^32.
+__host__ __device__ inline uint32_t div_small(uint32_t n, uint64_t inv) {
+  return static_cast<uint32_t>((static_cast<uint64_t>(n) * inv) >> 32);
+}
 
 // Valid tokens of cube c along each axis and in total.
 __host__ __device__ inline void cube_extent(const Geom& g, int c, int& nt, int& ny, int& nx,
                                             int& t0, int& y0, int& x0) {
-  int cx = c % g.Cx;
-  int r = c / g.Cx;
-  int cy = r % g.Cy;
-  int ct = r / g.Cy;
+  // c < kMaxCubes < 2^16, so the divisions by Cx and Cy use the reciprocals
+  const int r = static_cast<int>(div_small(static_cast<uint32_t>(c), g.inv_cx));
+  const int cx = c - r * g.Cx;
+  const int ct = static_cast<int>(div_small(static_cast<uint32_t>(r), g.inv_cy));
+  const int cy = r - ct * g.Cy;
   t0 = ct * 4; y0 = cy * 4; x0 = cx * 4;
   nt = min(4, g.T - t0);
   ny = min(4, g.Y - y0);

@@ -250,7 +250,12 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
   constexpr uint32_t kIdescQK128 = idesc_bf16_f32(64, 128, false, false);
   constexpr uint32_t kIdescQK64 = idesc_bf16_f32(64, 64, false, false);
   const uint32_t ring_base = smem_u32(sh.base + Cf::kRingOff);
-  uint32_t ring = 0;
+  // Ring position kept as (slot, phase) and advanced incrementally; the K and
+  // V descriptors of slot 0 are built once and a slot adds its byte offset / 16
+  // to the start-address field.
+  uint32_t slot_c = 0, phase_c = 0;
+  const uint64_t kdesc_base = sdesc_sw128(ring_base, 16, 1024);
+  const uint64_t vdesc_base = sdesc_sw128(ring_base, Cf::kKVHalf, 1024);
   uint32_t p_phase0 = 0u, p_phase1 = 0u;
   int t = 0;
   for (int item = blockIdx.x; item < items; item += gridDim.x, ++t) {
@@ -262,22 +267,22 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
     const uint32_t qa0 = smem_u32(sh.base + qb * 2 * Cf::kQBytes);
     const uint64_t qdesc0 = sdesc_sw128(qa0, 16, 1024);
     const uint64_t qdesc1 = sdesc_sw128(qa0 + Cf::kQBytes, 16, 1024);
-    auto next_slot = [&](uint32_t& addr) -> bool {
-      const uint32_t slot = ring % Cf::kSlots;
-      const uint32_t round = ring / Cf::kSlots;
-      ++ring;
-      if (!mbar_wait(&sh.kv_full[slot], round & 1u)) return false;
+    auto next_slot = [&](uint32_t& slot) -> bool {
+      slot = slot_c;
+      if (!mbar_wait(&sh.kv_full[slot], phase_c)) return false;
+      if (++slot_c == Cf::kSlots) {
+        slot_c = 0;
+        phase_c ^= 1u;
+      }
       tc_fence_after();
-      addr = ring_base + slot * Cf::kSlotBytes;
       return true;
     };
     // S_c = Q_c K^T over one step's keys
     auto qk = [&](int c, int j) -> bool {
-      uint32_t kb;
-      if (!next_slot(kb)) return false;
-      const uint32_t slot = (ring - 1) % Cf::kSlots;
+      uint32_t slot;
+      if (!next_slot(slot)) return false;
       const uint64_t a0 = c == 0 ? qdesc0 : qdesc1;
-      const uint64_t b0 = sdesc_sw128(kb, 16, 1024);
+      const uint64_t b0 = kdesc_base + (slot * Cf::kSlotBytes >> 4);
       const uint32_t idesc = (odd && j == nsteps - 1) ? kIdescQK64 : kIdescQK128;
       const uint32_t dS = tmem + (c == 0 ? Cf::kColS0 : Cf::kColS1);
 #pragma unroll
@@ -296,10 +301,9 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
       if (!mbar_wait(&sh.p_full[c], ph)) return false;
       ph ^= 1u;
       tc_fence_after();
-      uint32_t vb;
-      if (!next_slot(vb)) return false;
-      const uint32_t slot = (ring - 1) % Cf::kSlots;
-      const uint64_t v0 = sdesc_sw128(vb, Cf::kKVHalf, 1024);
+      uint32_t slot;
+      if (!next_slot(slot)) return false;
+      const uint64_t v0 = vdesc_base + (slot * Cf::kSlotBytes >> 4);
       const uint32_t dO = tmem + (c == 0 ? Cf::kColO0 : Cf::kColO1);
       const uint32_t aP = tmem + (c == 0 ? Cf::kColS0 : Cf::kColS1);
       const uint32_t acc0 = j > 0 ? 1u : 0u;
@@ -316,8 +320,9 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
     };
     if (!qk(0, 0)) return fail(sh, status);
     if (it.has_b && !qk(1, 0)) return fail(sh, status);
+    // No abort check inside the item: a failed role stops feeding this
+    // thread, whose next bounded wait then ends the item.
     for (int j = 0; j < nsteps; ++j) {
-      if (*sh.abort_flag) return;
       if (!pv(0, j)) return fail(sh, status);
       if (j + 1 < nsteps && !qk(0, j + 1)) return fail(sh, status);
       if (it.has_b) {

@@ -19,12 +19,19 @@ namespace {
 __device__ __forceinline__ long long slot_token(const Geom& g, int c, int s) {
   int nt, ny, nx, t0, y0, x0;
   cube_extent(g, c, nt, ny, nx, t0, y0, x0);
-  const int nyx = ny * nx;
-  if (s >= nt * nyx) return -1;
-  const int lt = s / nyx;
-  const int rem = s - lt * nyx;
-  const int ly = rem / nx;
-  const int lx = rem - ly * nx;
+  int lt, ly, lx;
+  if ((nt & ny & nx) == 4) {  // full cube: slot s = 16 lt + 4 ly + lx
+    lt = s >> 4;
+    ly = (s >> 2) & 3;
+    lx = s & 3;
+  } else {
+    const int nyx = ny * nx;
+    if (s >= nt * nyx) return -1;
+    lt = s / nyx;
+    const int rem = s - lt * nyx;
+    ly = rem / nx;
+    lx = rem - ly * nx;
+  }
   return (static_cast<long long>(t0 + lt) * g.Y + (y0 + ly)) * g.X + (x0 + lx);
 }
 
