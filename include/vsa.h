@@ -112,6 +112,18 @@ int vsa_coarse_select(const vsa_shape* shape, const void* q_tiled, const void* k
                       float* o_coarse, int32_t* sel_idx, float* coarse_logits,
                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* vsa_coarse_select on the TOKEN-ORDER tensors: the same result (pooled
+ * vectors, logits, selection, O_c) without waiting for vsa_tile_permute, so a
+ * caller can run the coarse stage on a second stream while q, k, v are tiled
+ * for the fine stage.  The pages have no counterpart: this is a scheduling
+ * convenience; the cube means are summed in the same row order as
+ * vsa_coarse_select, so both calls return identical bits.
+ *   q, k, v      bf16 [B, H, N, d] in token order
+ *   other arguments as vsa_coarse_select (no cube_count input) */
+int vsa_coarse_select_tokens(const vsa_shape* shape, const void* q, const void* k, const void* v,
+                             int topk, float* o_coarse, int32_t* sel_idx, float* coarse_logits,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* vsa_coarse_select for callers that cannot allocate device memory.  The
  * pages have no counterpart: this is a library convenience.  Some callers own
  * no device allocator (a plugin inside a host application that manages all

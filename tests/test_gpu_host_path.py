@@ -3,7 +3,8 @@
 same kernels as the device-buffer path, so the output must equal that path's
 bit for bit (the device path itself is checked against the oracle in
 test_gpu_parity.py); chunk sizes that do not divide B*H, and chunks that
-cross a batch boundary, are covered."""
+cross a batch boundary, are covered.  The device-buffer path is also replayed
+from a captured CUDA graph."""
 
 import numpy as np
 import pytest
@@ -80,3 +81,31 @@ def test_host_path_reuses_its_workspace(vsa):
     shape = vsa.make_shape(w.batch, w.heads, w.head_dim, w.grid)
     a, b = host_path(vsa, w, x, shape, 4, repeats=2)
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_device_path_replays_from_a_cuda_graph(vsa):
+    # after one eager call the path only launches kernels, so a stream capture
+    # of it replays to the same bits
+    w = wl.WORKLOADS["wan1.3b_ft_16x28x52"]
+    x = wl.make_inputs(w)
+    shape = vsa.make_shape(w.batch, w.heads, w.head_dim, w.grid)
+    q, k, v = (to_dev_bf16(x[n]) for n in ("q", "k", "v"))
+    g_f = torch.from_numpy(x["g_f"]).cuda()
+    g_c = torch.from_numpy(x["g_c"]).cuda()
+    out_eager = torch.empty_like(q)
+    bufs = vsa.vsa_forward(shape, q, k, v, w.topk, out_eager, g_f, g_c)
+    torch.cuda.synchronize()
+    out_graph = torch.zeros_like(q)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            vsa.vsa_forward(shape, q, k, v, w.topk, out_graph, g_f, g_c, bufs=bufs)
+    for _ in range(2):
+        out_graph.zero_()
+        graph.replay()
+    torch.cuda.synchronize()
+    assert vsa.vsa_get_status() == 0
+    assert torch.equal(out_graph.view(torch.int16), out_eager.view(torch.int16))
+    del graph

@@ -117,6 +117,26 @@ def test_coarse_select(vsa, B, H, d, grid, k):
     assert vsa.vsa_get_status() == 0
 
 
+@pytest.mark.parametrize("B,H,d,grid,k", [(1, 2, 64, (4, 8, 8), 2), (2, 3, 128, (9, 10, 11), 5),
+                                           (1, 2, 128, (21, 30, 52), 62)])
+def test_coarse_select_tokens_equals_tiled_call(vsa, B, H, d, grid, k):
+    # pooling straight from token order sums each cube's rows in the same order
+    w, x, shape, C, bufs, logits = coarse_run(vsa, B, H, d, grid, k)
+    sel = torch.empty_like(bufs.sel)
+    o_c = torch.empty_like(bufs.o_c)
+    lg = torch.empty_like(logits)
+    ws = torch.empty_like(bufs.workspace)
+    vsa.vsa_coarse_select_tokens(shape, to_dev_bf16(x["q"]), to_dev_bf16(x["k"]), to_dev_bf16(x["v"]),
+                                 k, sel, ws, o_coarse=o_c, coarse_logits=lg)
+    torch.cuda.synchronize()
+    assert vsa.vsa_get_status() == 0
+    n = 3 * B * H * C * d * 4
+    assert torch.equal(ws[:n], bufs.workspace[:n])
+    assert torch.equal(lg, logits)
+    assert torch.equal(sel, bufs.sel)
+    assert torch.equal(o_c, bufs.o_c)
+
+
 @pytest.mark.parametrize("grid,k", [((8, 8, 8), 3), ((48, 48, 48), 1700)])
 def test_topk_ties_go_to_lower_index(vsa, grid, k):
     # identical k vectors in every cube -> all coarse logits of a row tie

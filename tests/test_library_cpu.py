@@ -88,6 +88,12 @@ def test_null_and_misaligned_pointers_rejected_before_launch(vsa):
     assert lib.vsa_coarse_select(ctypes.byref(s), p, p, p, p, 2, None, p, None, p, 16, None) == vsa.VSA_ERR_INVALID_ARG
     # one gate without the other
     assert lib.vsa_combine(ctypes.byref(s), p, p, p, None, p, None) == vsa.VSA_ERR_INVALID_ARG
+    # token-order coarse stage: k out of range, missing output, small or misaligned workspace
+    tok = lib.vsa_coarse_select_tokens
+    assert tok(ctypes.byref(s), p, p, p, 5, None, p, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
+    assert tok(ctypes.byref(s), p, p, p, 2, None, None, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
+    assert tok(ctypes.byref(s), p, p, p, 2, None, p, None, p, 16, None) == vsa.VSA_ERR_INVALID_ARG
+    assert tok(ctypes.byref(s), odd, p, p, 2, None, p, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
     assert lib.vsa_debug_wait_timeout(10, None) == vsa.VSA_ERR_INVALID_ARG
 
 

@@ -18,7 +18,7 @@ cudaError_t launch_combine(const Geom&, const void*, const float*, const float*,
                            void*, int, cudaStream_t);
 cudaError_t launch_coarse_select(const Geom&, const void*, const void*, const void*,
                                  const int32_t*, int, float*, int32_t*, float*, float*, int*,
-                                 cudaStream_t);
+                                 cudaStream_t, bool token_order);
 cudaError_t launch_block_sparse_fwd(const Geom&, const CUtensorMap&, const CUtensorMap&,
                                     const CUtensorMap&, const int32_t*, const int32_t*, int,
                                     void*, float*, int*, int, cudaStream_t);
@@ -229,7 +229,27 @@ int vsa_coarse_select(const vsa_shape* shape, const void* q_tiled, const void* k
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_coarse_select(g, q_tiled, k_tiled, v_tiled, cube_count, topk, o_coarse,
                                       sel_idx, coarse_logits, static_cast<float*>(workspace),
-                                      st->status, stream));
+                                      st->status, stream, false));
+}
+
+int vsa_coarse_select_tokens(const vsa_shape* shape, const void* q, const void* k, const void* v,
+                             int topk, float* o_coarse, int32_t* sel_idx, float* coarse_logits,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (topk < 1 || topk > g.C) return VSA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !sel_idx || !workspace) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (reinterpret_cast<uintptr_t>(sel_idx) & 3u) || (o_coarse && !aligned16(o_coarse)) ||
+      (coarse_logits && (reinterpret_cast<uintptr_t>(coarse_logits) & 3u)))
+    return VSA_ERR_INVALID_ARG;
+  if (workspace_bytes < vsa_workspace_bytes(shape, topk)) return VSA_ERR_INVALID_ARG;
+  DeviceState* st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  return cuda_rc(launch_coarse_select(g, q, k, v, nullptr, topk, o_coarse, sel_idx, coarse_logits,
+                                      static_cast<float*>(workspace), st->status, stream, true));
 }
 
 int vsa_block_sparse_fwd(const vsa_shape* shape, const void* q_tiled, const void* k_tiled,

@@ -3,7 +3,8 @@
 // section "传统零散郑重力，为何会在蒸馏中失效？").
 //
 // 1. pool_kernel: qbar, kbar, vbar = mean of each cube's n_c valid rows
-//    (float32), an HBM-bound pass over the three tiled tensors.
+//    (float32), an HBM-bound pass over the three tiled tensors, or over the
+//    token-order tensors (so the coarse stage need not wait for the tiling).
 // 2. coarse_kernel: for a tile of R query cubes of one (b, h):
 //      S_c[i, :] = qbar_i kbar^T / sqrt(d)       (float32, row kept in smem)
 //      sel[i]    = top-k of S_c[i, :], ties to the lower index, ascending
@@ -31,7 +32,8 @@ __global__ void __launch_bounds__(256) pool_kernel(Geom g, const uint4* __restri
                                                    const uint4* __restrict__ k,
                                                    const uint4* __restrict__ v,
                                                    const int32_t* __restrict__ counts,
-                                                   float* __restrict__ ws, int* status) {
+                                                   float* __restrict__ ws, int* status,
+                                                   bool token_order) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long item = static_cast<long long>(blockIdx.x) * 8 + warp;  // (b*h, cube)
   const long long items = static_cast<long long>(g.B) * g.H * g.C;
@@ -41,16 +43,21 @@ __global__ void __launch_bounds__(256) pool_kernel(Geom g, const uint4* __restri
   const long long bh = item / g.C;
   const int c = static_cast<int>(item - bh * g.C);
   const int n = cube_valid(g, c);
-  if (which == 0 && lane == 0 && counts[c] != n) report(status, VSA_ERR_BAD_INDEX);
+  if (which == 0 && lane == 0 && counts != nullptr && counts[c] != n)
+    report(status, VSA_ERR_BAD_INDEX);
 
   const int chunks = g.d >> 3;         // 8 or 16
   const int rows_per_step = 32 / chunks;  // 4 or 2
   const int ch = lane % chunks;
   const int r0 = lane / chunks;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  const uint4* base = src + (bh * g.rows + static_cast<long long>(c) * kSlots) * chunks;
+  // tiled input: the cube's valid rows are its first n rows; token-order input:
+  // row r of the cube is token slot_token(c, r) of the (b, h) plane
+  const uint4* base = token_order ? src + bh * g.N * chunks
+                                  : src + (bh * g.rows + static_cast<long long>(c) * kSlots) * chunks;
   for (int r = r0; r < n; r += rows_per_step) {
-    const uint4 w = __ldg(&base[static_cast<long long>(r) * chunks + ch]);
+    const long long row = token_order ? slot_token(g, c, r) : r;
+    const uint4 w = __ldg(&base[row * chunks + ch]);
     const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -372,18 +379,24 @@ size_t coarse_smem_bytes(int C, int d, int R) {
 cudaError_t launch_coarse_select(const Geom& g, const void* qt, const void* kt, const void* vt,
                                  const int32_t* counts, int topk, float* o_coarse,
                                  int32_t* sel, float* logits, float* ws, int* status,
-                                 cudaStream_t s) {
+                                 cudaStream_t s, bool token_order) {
   const long long items = static_cast<long long>(g.B) * g.H * g.C;
   dim3 pg(static_cast<unsigned>((items + 7) / 8), 3);
   pool_kernel<<<pg, 256, 0, s>>>(g, static_cast<const uint4*>(qt), static_cast<const uint4*>(kt),
-                                 static_cast<const uint4*>(vt), counts, ws, status);
+                                 static_cast<const uint4*>(vt), counts, ws, status, token_order);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const int R = coarse_rows_per_cta(g.C, g.d);
   const size_t smem = coarse_smem_bytes(g.C, g.d, R);
-  err = cudaFuncSetAttribute(coarse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
+  // the limit is raised once per device to the largest block any accepted
+  // shape needs: the logits block never exceeds kLogitBudgetBytes, plus qT
+  // for d = 128, the staging buffer and the top-k histograms
+  static unsigned long long limit_set = 0;
+  const size_t most = kLogitBudgetBytes + (static_cast<size_t>(128) * 16 + kStageFloats) * sizeof(float) +
+                      8 * 256 * sizeof(int);
+  err = smem_limit_once(coarse_kernel, static_cast<int>(most), &limit_set);
   if (err != cudaSuccess) return err;
+  if (smem > most) return cudaErrorInvalidValue;
   dim3 cg(static_cast<unsigned>((g.C + R - 1) / R), static_cast<unsigned>(g.B * g.H));
   coarse_kernel<<<cg, kCoarseThreads, smem, s>>>(g, R, topk, ws, o_coarse, sel, logits);
   return cudaGetLastError();

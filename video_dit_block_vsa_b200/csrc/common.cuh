@@ -53,6 +53,41 @@ __host__ __device__ inline int cube_valid(const Geom& g, int c) {
   return nt * ny * nx;
 }
 
+// Token index held by slot s of cube c, or -1 for a pad slot.
+__device__ __forceinline__ long long slot_token(const Geom& g, int c, int s) {
+  int nt, ny, nx, t0, y0, x0;
+  cube_extent(g, c, nt, ny, nx, t0, y0, x0);
+  int lt, ly, lx;
+  if ((nt & ny & nx) == 4) {  // full cube: slot s = 16 lt + 4 ly + lx
+    lt = s >> 4;
+    ly = (s >> 2) & 3;
+    lx = s & 3;
+  } else {
+    const int nyx = ny * nx;
+    if (s >= nt * nyx) return -1;
+    lt = s / nyx;
+    const int rem = s - lt * nyx;
+    ly = rem / nx;
+    lx = rem - ly * nx;
+  }
+  return (static_cast<long long>(t0 + lt) * g.Y + (y0 + ly)) * g.X + (x0 + lx);
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device (bit d of
+// *done for device d), so that later launches, including launches made
+// while a stream is being captured into a CUDA graph, only launch.
+template <typename Kernel>
+inline cudaError_t smem_limit_once(Kernel kernel, int bytes, unsigned long long* done) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (__atomic_load_n(done, __ATOMIC_ACQUIRE) & bit) return cudaSuccess;
+  err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err == cudaSuccess) __atomic_fetch_or(done, bit, __ATOMIC_RELEASE);
+  return err;
+}
+
 // Record a device-side condition in the status word (first one wins).
 __device__ inline void report(int* status, int code) {
   if (status) atomicCAS(status, 0, code);

@@ -540,15 +540,14 @@ cudaError_t launch_block_sparse_fwd(const Geom& g, const CUtensorMap& tq, const 
   const int grid = static_cast<int>(items < sms ? items : sms);
   const size_t smem = fine_smem_bytes(g.d);
   cudaError_t err;
+  static unsigned long long limit_set[2] = {0, 0};
   if (g.d == 128) {
-    err = cudaFuncSetAttribute(fine_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
+    err = smem_limit_once(fine_fwd_kernel<128>, static_cast<int>(smem), &limit_set[0]);
     if (err != cudaSuccess) return err;
     fine_fwd_kernel<128><<<grid, kThreads, smem, s>>>(tq, tk, tv, g, counts, sel, topk,
                                                        static_cast<__nv_bfloat16*>(out), lse, status);
   } else {
-    err = cudaFuncSetAttribute(fine_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
+    err = smem_limit_once(fine_fwd_kernel<64>, static_cast<int>(smem), &limit_set[1]);
     if (err != cudaSuccess) return err;
     fine_fwd_kernel<64><<<grid, kThreads, smem, s>>>(tq, tk, tv, g, counts, sel, topk,
                                                       static_cast<__nv_bfloat16*>(out), lse, status);

@@ -15,26 +15,6 @@ namespace vsa {
 
 namespace {
 
-// Token index held by slot s of cube c, or -1 for a pad slot.
-__device__ __forceinline__ long long slot_token(const Geom& g, int c, int s) {
-  int nt, ny, nx, t0, y0, x0;
-  cube_extent(g, c, nt, ny, nx, t0, y0, x0);
-  int lt, ly, lx;
-  if ((nt & ny & nx) == 4) {  // full cube: slot s = 16 lt + 4 ly + lx
-    lt = s >> 4;
-    ly = (s >> 2) & 3;
-    lx = s & 3;
-  } else {
-    const int nyx = ny * nx;
-    if (s >= nt * nyx) return -1;
-    lt = s / nyx;
-    const int rem = s - lt * nyx;
-    ly = rem / nx;
-    lx = rem - ly * nx;
-  }
-  return (static_cast<long long>(t0 + lt) * g.Y + (y0 + ly)) * g.X + (x0 + lx);
-}
-
 __global__ void __launch_bounds__(256) tile_permute_kernel(Geom g, const uint4* __restrict__ x,
                                                            uint4* __restrict__ xt,
                                                            int32_t* __restrict__ counts) {
