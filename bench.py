@@ -4,9 +4,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
 A step is one pass of the whole path over one batch: tile q, k, v into
-cubes; coarse stage (pool, coarse attention, top-k), which pools straight
-from the token-order inputs on a second stream and so overlaps the tiling;
-fine block-sparse attention; gated combine; untile.  Inputs are drawn once on the host from the
+cubes and pool them per cube (one pass over the inputs); coarse attention and
+top-k; fine block-sparse attention; gated combine; untile.  Inputs are drawn once on the host from the
 seeded synthetic recipe and are resident in HBM before the timed region; each
 input tensor (774 MB at the default workload) is larger than the 126 MB L2,
 so no flush is needed between steps.
@@ -251,30 +250,16 @@ def run_gpu(args, w):
     bufs = vsa.VsaBuffers(shape, w.topk, device=dev, want_coarse=w.gated)
     stream = torch.cuda.current_stream()
 
-    # The coarse stage pools straight from the token-order inputs on a second
-    # stream, so it overlaps the three tiling passes (HBM-bound) instead of
-    # waiting for them; the fine stage waits for both.
-    side = torch.cuda.Stream(dev)
-    fork = torch.cuda.Event()
-    join = torch.cuda.Event()
-
     def step(ev=None):
-        def mark(i, st=stream):
+        def mark(i):
             if ev is not None:
-                ev[i].record(st)
+                ev[i].record(stream)
         mark(0)
-        fork.record(stream)
-        side.wait_event(fork)
-        mark(6, side)
-        vsa.vsa_coarse_select_tokens(shape, q, k, v, w.topk, bufs.sel, bufs.workspace,
-                                     o_coarse=bufs.o_c, stream=side)
-        mark(7, side)
-        join.record(side)
-        vsa.vsa_tile_permute(shape, q, bufs.q_t, bufs.counts)
-        vsa.vsa_tile_permute(shape, k, bufs.k_t)
-        vsa.vsa_tile_permute(shape, v, bufs.v_t)
+        # one pass over q, k, v: tiled copies plus the cube means of the coarse stage
+        vsa.vsa_tile_permute_pool(shape, q, k, v, bufs.q_t, bufs.k_t, bufs.v_t, bufs.workspace,
+                                  bufs.counts)
         mark(1)
-        stream.wait_event(join)
+        vsa.vsa_coarse_select_pooled(shape, w.topk, bufs.sel, bufs.workspace, o_coarse=bufs.o_c)
         mark(2)
         vsa.vsa_block_sparse_fwd(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, bufs.sel,
                                  w.topk, bufs.o_f)
@@ -284,7 +269,7 @@ def run_gpu(args, w):
         vsa.vsa_untile(shape, bufs.o_f, out)
         mark(5)
 
-    launches_per_step = 3 + 2 + 1 + (1 if w.gated else 0) + 1
+    launches_per_step = 1 + 1 + 1 + (1 if w.gated else 0) + 1
 
     for _ in range(max(args.warmup, 1)):
         step()
@@ -296,7 +281,7 @@ def run_gpu(args, w):
     fine_eff, fine_issued, coarse_fl = flop_counts(w, counts, bufs.sel.cpu().numpy().astype(np.int64))
     step_flops = fine_eff + coarse_fl
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     vdist.barrier(ri)
     torch.cuda.synchronize()
@@ -314,11 +299,10 @@ def run_gpu(args, w):
     status = vsa.vsa_get_status()
     if status != 0:
         raise RuntimeError(f"device status after timed steps: {vsa.vsa_strerror(status)}")
-    # event pairs per stage: the coarse stage runs on the side stream (6 -> 7),
-    # concurrently with the tiling (0 -> 1); "coarse_wait" is the time the fine
-    # stage still waited for it after the tiling (1 -> 2)
-    pairs = {"tile_permute": (0, 1), "coarse_select": (6, 7), "coarse_wait": (1, 2),
-             "block_sparse_fwd": (2, 3), "combine": (3, 4), "untile": (4, 5)}
+    # stage "tile_permute" is the one pass that tiles q, k, v and pools them;
+    # "coarse_select" is the coarse attention, top-k and O_c from those means
+    pairs = {"tile_permute": (0, 1), "coarse_select": (1, 2), "block_sparse_fwd": (2, 3),
+             "combine": (3, 4), "untile": (4, 5)}
     stage_ms = {name: statistics.mean(evs[s][a_].elapsed_time(evs[s][b_]) for s in range(args.steps))
                 for name, (a_, b_) in pairs.items()}
     ms_per_step = elapsed_ms / args.steps
@@ -396,7 +380,10 @@ def run_gpu(args, w):
             cpu["s_per_call_extrapolated"] = sum(per_head.values()) * w.batch * w.heads
 
     if rank == 0:
-        hbm_bytes = {  # passes timed alone (tile_permute overlaps the coarse stage)
+        hbm_bytes = {
+            # read q, k, v once; write the tiled copies and the float32 cube means
+            "tile_permute": (3 * w.batch * w.heads * (w.tokens + 64 * w.cubes) * w.head_dim * 2
+                             + 3 * w.batch * w.heads * w.cubes * w.head_dim * 4),
             "untile": w.batch * w.heads * 2 * w.tokens * w.head_dim * 2,  # valid rows in, tokens out
         }
         line = {
@@ -414,9 +401,8 @@ def run_gpu(args, w):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
             "stages_ms": stage_ms,
-            "stages_note": ("coarse_select runs on a second stream while tile_permute runs, so "
-                            "those two times overlap and include each other's contention; "
-                            "coarse_wait is what the fine stage still waited for it"),
+            "stages_note": ("tile_permute is one pass that tiles q, k, v and writes their cube "
+                            "means (the coarse stage's pooling); coarse_select starts from those"),
             "stages_gbs": {k: v / (stage_ms[k] * 1e-3) / 1e9 for k, v in hbm_bytes.items()},
             "flops": {"fine_effective": fine_eff, "fine_issued": fine_issued, "coarse": coarse_fl},
             "kernel_rev": KERNEL_REV,

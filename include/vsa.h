@@ -112,6 +112,28 @@ int vsa_coarse_select(const vsa_shape* shape, const void* q_tiled, const void* k
                       float* o_coarse, int32_t* sel_idx, float* coarse_logits,
                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Tiling and pooling in one pass over q, k, v: writes q_tiled, k_tiled,
+ * v_tiled and cube_count exactly as three vsa_tile_permute calls, and the
+ * per-cube means (float32, the first 3*B*H*C*d*4 bytes of the workspace, in
+ * the layout vsa_coarse_select uses) exactly as vsa_coarse_select's pooling,
+ * so each input tensor is read once.  The pages have no counterpart: this is
+ * the coarse stage's pooling fused into the tiling pass.
+ *   q, k, v          bf16 [B, H, N, d] token order
+ *   *_tiled          bf16 [B, H, 64*C, d] (written)
+ *   cube_count       int32 [C] or NULL (written)
+ *   workspace        >= vsa_workspace_bytes(shape, 1) bytes, 256-byte aligned */
+int vsa_tile_permute_pool(const vsa_shape* shape, const void* q, const void* k, const void* v,
+                          void* q_tiled, void* k_tiled, void* v_tiled, int32_t* cube_count,
+                          void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* The coarse stage after vsa_tile_permute_pool: coarse attention, top-k and
+ * O_c from the cube means already in `workspace` (same outputs, bit for bit,
+ * as vsa_coarse_select on the tiled tensors).  Arguments as vsa_coarse_select
+ * minus the tensors. */
+int vsa_coarse_select_pooled(const vsa_shape* shape, int topk, float* o_coarse, int32_t* sel_idx,
+                             float* coarse_logits, const void* workspace, size_t workspace_bytes,
+                             cudaStream_t stream);
+
 /* vsa_coarse_select on the TOKEN-ORDER tensors: the same result (pooled
  * vectors, logits, selection, O_c) without waiting for vsa_tile_permute, so a
  * caller can run the coarse stage on a second stream while q, k, v are tiled

@@ -137,6 +137,33 @@ def test_coarse_select_tokens_equals_tiled_call(vsa, B, H, d, grid, k):
     assert torch.equal(o_c, bufs.o_c)
 
 
+@pytest.mark.parametrize("B,H,d,grid,k", [(1, 2, 64, (4, 8, 8), 2), (2, 3, 128, (9, 10, 11), 5),
+                                           (1, 2, 128, (21, 30, 52), 62), (1, 1, 64, (1, 1, 1), 1)])
+def test_fused_tile_pool_equals_separate_calls(vsa, B, H, d, grid, k):
+    # one pass that tiles q, k, v and pools them gives the same bits as the
+    # three tiling calls plus the coarse call's own pooling
+    w, x, shape, C, bufs, logits = coarse_run(vsa, B, H, d, grid, k)
+    qt, kt, vt = (torch.full_like(bufs.q_t, 7.0) for _ in range(3))  # pads must be overwritten
+    counts = torch.full_like(bufs.counts, -1)
+    ws = torch.empty_like(bufs.workspace)
+    vsa.vsa_tile_permute_pool(shape, to_dev_bf16(x["q"]), to_dev_bf16(x["k"]), to_dev_bf16(x["v"]),
+                              qt, kt, vt, ws, counts)
+    sel = torch.empty_like(bufs.sel)
+    o_c = torch.empty_like(bufs.o_c)
+    lg = torch.empty_like(logits)
+    vsa.vsa_coarse_select_pooled(shape, k, sel, ws, o_coarse=o_c, coarse_logits=lg)
+    torch.cuda.synchronize()
+    assert vsa.vsa_get_status() == 0
+    for got, want in ((qt, bufs.q_t), (kt, bufs.k_t), (vt, bufs.v_t)):
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+    assert torch.equal(counts, bufs.counts)
+    n = 3 * B * H * C * d * 4
+    assert torch.equal(ws[:n], bufs.workspace[:n])
+    assert torch.equal(lg, logits)
+    assert torch.equal(sel, bufs.sel)
+    assert torch.equal(o_c, bufs.o_c)
+
+
 @pytest.mark.parametrize("grid,k", [((8, 8, 8), 3), ((48, 48, 48), 1700)])
 def test_topk_ties_go_to_lower_index(vsa, grid, k):
     # identical k vectors in every cube -> all coarse logits of a row tie

@@ -94,6 +94,15 @@ def test_null_and_misaligned_pointers_rejected_before_launch(vsa):
     assert tok(ctypes.byref(s), p, p, p, 2, None, None, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
     assert tok(ctypes.byref(s), p, p, p, 2, None, p, None, p, 16, None) == vsa.VSA_ERR_INVALID_ARG
     assert tok(ctypes.byref(s), odd, p, p, 2, None, p, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
+    # fused tiling + pooling, and the coarse stage from pooled means
+    tp = lib.vsa_tile_permute_pool
+    assert tp(ctypes.byref(s), p, p, p, p, p, None, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
+    assert tp(ctypes.byref(s), p, p, p, p, p, p, None, p, 16, None) == vsa.VSA_ERR_INVALID_ARG
+    assert tp(ctypes.byref(s), p, odd, p, p, p, p, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
+    cp = lib.vsa_coarse_select_pooled
+    assert cp(ctypes.byref(s), 5, None, p, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
+    assert cp(ctypes.byref(s), 2, None, None, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
+    assert cp(ctypes.byref(s), 2, None, p, None, p, 16, None) == vsa.VSA_ERR_INVALID_ARG
     assert lib.vsa_debug_wait_timeout(10, None) == vsa.VSA_ERR_INVALID_ARG
 
 

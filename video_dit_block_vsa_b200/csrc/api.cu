@@ -19,6 +19,10 @@ cudaError_t launch_combine(const Geom&, const void*, const float*, const float*,
 cudaError_t launch_coarse_select(const Geom&, const void*, const void*, const void*,
                                  const int32_t*, int, float*, int32_t*, float*, float*, int*,
                                  cudaStream_t, bool token_order);
+cudaError_t launch_tile_pool(const Geom&, const void*, const void*, const void*, void*, void*,
+                             void*, int32_t*, float*, int*, cudaStream_t);
+cudaError_t launch_coarse_only(const Geom&, int, float*, int32_t*, float*, const float*,
+                               cudaStream_t);
 cudaError_t launch_block_sparse_fwd(const Geom&, const CUtensorMap&, const CUtensorMap&,
                                     const CUtensorMap&, const int32_t*, const int32_t*, int,
                                     void*, float*, int*, int, cudaStream_t);
@@ -230,6 +234,44 @@ int vsa_coarse_select(const vsa_shape* shape, const void* q_tiled, const void* k
   return cuda_rc(launch_coarse_select(g, q_tiled, k_tiled, v_tiled, cube_count, topk, o_coarse,
                                       sel_idx, coarse_logits, static_cast<float*>(workspace),
                                       st->status, stream, false));
+}
+
+int vsa_tile_permute_pool(const vsa_shape* shape, const void* q, const void* k, const void* v,
+                          void* q_tiled, void* k_tiled, void* v_tiled, int32_t* cube_count,
+                          void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (!q || !k || !v || !q_tiled || !k_tiled || !v_tiled || !workspace) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_tiled) ||
+      !aligned16(k_tiled) || !aligned16(v_tiled) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (cube_count && (reinterpret_cast<uintptr_t>(cube_count) & 3u)))
+    return VSA_ERR_INVALID_ARG;
+  if (workspace_bytes < vsa_workspace_bytes(shape, 1)) return VSA_ERR_INVALID_ARG;
+  DeviceState* st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  return cuda_rc(launch_tile_pool(g, q, k, v, q_tiled, k_tiled, v_tiled, cube_count,
+                                  static_cast<float*>(workspace), st->status, stream));
+}
+
+int vsa_coarse_select_pooled(const vsa_shape* shape, int topk, float* o_coarse, int32_t* sel_idx,
+                             float* coarse_logits, const void* workspace, size_t workspace_bytes,
+                             cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (topk < 1 || topk > g.C) return VSA_ERR_INVALID_ARG;
+  if (!sel_idx || !workspace) return VSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (reinterpret_cast<uintptr_t>(sel_idx) & 3u) || (o_coarse && !aligned16(o_coarse)) ||
+      (coarse_logits && (reinterpret_cast<uintptr_t>(coarse_logits) & 3u)))
+    return VSA_ERR_INVALID_ARG;
+  if (workspace_bytes < vsa_workspace_bytes(shape, topk)) return VSA_ERR_INVALID_ARG;
+  DeviceState* st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  return cuda_rc(launch_coarse_only(g, topk, o_coarse, sel_idx, coarse_logits,
+                                    static_cast<const float*>(workspace), stream));
 }
 
 int vsa_coarse_select_tokens(const vsa_shape* shape, const void* q, const void* k, const void* v,

@@ -28,12 +28,18 @@ constexpr int kLogitBudgetBytes = 132 * 1024;
 // ------------------------------------------------------------------ pooling
 // One warp per (tensor, b*h, cube).  A row of d bf16 is d/8 16-byte chunks;
 // the warp covers 32/(d/8) rows per step and reduces across row groups at the end.
+// With token-order input and tiled outputs given, the same pass also writes the
+// tiled tensors (valid rows copied, pad rows zero) and the cube counts: the
+// tiling and the pooling then cost one read of q, k, v.
 __global__ void __launch_bounds__(256) pool_kernel(Geom g, const uint4* __restrict__ q,
                                                    const uint4* __restrict__ k,
                                                    const uint4* __restrict__ v,
                                                    const int32_t* __restrict__ counts,
                                                    float* __restrict__ ws, int* status,
-                                                   bool token_order) {
+                                                   bool token_order, uint4* __restrict__ qt,
+                                                   uint4* __restrict__ kt,
+                                                   uint4* __restrict__ vt,
+                                                   int32_t* __restrict__ counts_out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long item = static_cast<long long>(blockIdx.x) * 8 + warp;  // (b*h, cube)
   const long long items = static_cast<long long>(g.B) * g.H * g.C;
@@ -55,15 +61,24 @@ __global__ void __launch_bounds__(256) pool_kernel(Geom g, const uint4* __restri
   // row r of the cube is token slot_token(c, r) of the (b, h) plane
   const uint4* base = token_order ? src + bh * g.N * chunks
                                   : src + (bh * g.rows + static_cast<long long>(c) * kSlots) * chunks;
+  uint4* tiled = which == 0 ? qt : (which == 1 ? kt : vt);
+  if (tiled != nullptr) tiled += (bh * g.rows + static_cast<long long>(c) * kSlots) * chunks;
+  if (counts_out != nullptr && which == 0 && bh == 0 && lane == 0) counts_out[c] = n;
+#pragma unroll 4
   for (int r = r0; r < n; r += rows_per_step) {
     const long long row = token_order ? slot_token(g, c, r) : r;
     const uint4 w = __ldg(&base[row * chunks + ch]);
+    if (tiled != nullptr) tiled[r * chunks + ch] = w;
     const uint32_t u[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       acc[2 * e] += __uint_as_float(u[e] << 16);
       acc[2 * e + 1] += __uint_as_float(u[e] & 0xFFFF0000u);
     }
+  }
+  if (tiled != nullptr) {  // pad rows of the tiled copy
+    for (int r = r0; r < kSlots; r += rows_per_step)
+      if (r >= n) tiled[r * chunks + ch] = make_uint4(0u, 0u, 0u, 0u);
   }
   for (int off = chunks; off < 32; off <<= 1) {
 #pragma unroll
@@ -376,6 +391,9 @@ size_t coarse_smem_bytes(int C, int d, int R) {
              sizeof(float) + 8 * 256 * sizeof(int);
 }
 
+cudaError_t launch_coarse_only(const Geom& g, int topk, float* o_coarse, int32_t* sel,
+                               float* logits, const float* ws, cudaStream_t s);
+
 cudaError_t launch_coarse_select(const Geom& g, const void* qt, const void* kt, const void* vt,
                                  const int32_t* counts, int topk, float* o_coarse,
                                  int32_t* sel, float* logits, float* ws, int* status,
@@ -383,9 +401,28 @@ cudaError_t launch_coarse_select(const Geom& g, const void* qt, const void* kt, 
   const long long items = static_cast<long long>(g.B) * g.H * g.C;
   dim3 pg(static_cast<unsigned>((items + 7) / 8), 3);
   pool_kernel<<<pg, 256, 0, s>>>(g, static_cast<const uint4*>(qt), static_cast<const uint4*>(kt),
-                                 static_cast<const uint4*>(vt), counts, ws, status, token_order);
+                                 static_cast<const uint4*>(vt), counts, ws, status, token_order,
+                                 nullptr, nullptr, nullptr, nullptr);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
+  return launch_coarse_only(g, topk, o_coarse, sel, logits, ws, s);
+}
+
+cudaError_t launch_tile_pool(const Geom& g, const void* q, const void* k, const void* v,
+                             void* qt, void* kt, void* vt, int32_t* counts, float* ws,
+                             int* status, cudaStream_t s) {
+  const long long items = static_cast<long long>(g.B) * g.H * g.C;
+  dim3 pg(static_cast<unsigned>((items + 7) / 8), 3);
+  pool_kernel<<<pg, 256, 0, s>>>(g, static_cast<const uint4*>(q), static_cast<const uint4*>(k),
+                                 static_cast<const uint4*>(v), nullptr, ws, status, true,
+                                 static_cast<uint4*>(qt), static_cast<uint4*>(kt),
+                                 static_cast<uint4*>(vt), counts);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_coarse_only(const Geom& g, int topk, float* o_coarse, int32_t* sel,
+                               float* logits, const float* ws, cudaStream_t s) {
+  cudaError_t err;
   const int R = coarse_rows_per_cta(g.C, g.d);
   const size_t smem = coarse_smem_bytes(g.C, g.d, R);
   // the limit is raised once per device to the largest block any accepted

@@ -3,7 +3,9 @@
 // computes on the caller's stream, the next chunk's q, k, v (and gates) are
 // copied in on one internal stream and the previous chunk's output is copied
 // out on another, so PCIe transfers in both directions overlap the kernels.
-// Every stage runs through the same entry points as the device-buffer path.
+// Every stage runs through the same entry points as the device-buffer path
+// (tiling and pooling in one pass, then the coarse stage, fine stage, combine
+// and untile).
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -182,11 +184,11 @@ int vsa_forward_host(const vsa_shape* shape, int topk, const void* q, const void
     int32_t* sel = reinterpret_cast<int32_t*>(base + L.sel);
     float* oc = gated ? reinterpret_cast<float*>(base + L.oc) : nullptr;
     const size_t pool_bytes = vsa_workspace_bytes(&sub, topk);
-    if ((rc = vsa_tile_permute(&sub, base + L.x[0], base + L.xt[0], counts, stream)) != VSA_OK ||
-        (rc = vsa_tile_permute(&sub, base + L.x[1], base + L.xt[1], nullptr, stream)) != VSA_OK ||
-        (rc = vsa_tile_permute(&sub, base + L.x[2], base + L.xt[2], nullptr, stream)) != VSA_OK ||
-        (rc = vsa_coarse_select(&sub, base + L.xt[0], base + L.xt[1], base + L.xt[2], counts, topk,
-                                oc, sel, nullptr, base + L.pool, pool_bytes, stream)) != VSA_OK ||
+    if ((rc = vsa_tile_permute_pool(&sub, base + L.x[0], base + L.x[1], base + L.x[2],
+                                    base + L.xt[0], base + L.xt[1], base + L.xt[2], counts,
+                                    base + L.pool, pool_bytes, stream)) != VSA_OK ||
+        (rc = vsa_coarse_select_pooled(&sub, topk, oc, sel, nullptr, base + L.pool, pool_bytes,
+                                       stream)) != VSA_OK ||
         (rc = vsa_block_sparse_fwd(&sub, base + L.xt[0], base + L.xt[1], base + L.xt[2], counts,
                                    sel, topk, base + L.of, nullptr, stream)) != VSA_OK ||
         (rc = vsa_combine(&sub, base + L.of, oc,

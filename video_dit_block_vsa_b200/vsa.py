@@ -32,7 +32,8 @@ VSA_ERR_BAD_INDEX = 5
 VSA_ERR_TOO_LARGE = 6
 
 EXPORTED = ("vsa_num_cubes", "vsa_topk_from_ratio", "vsa_workspace_bytes", "vsa_tile_permute",
-            "vsa_coarse_select", "vsa_coarse_select_tokens", "vsa_coarse_select_noalloc",
+            "vsa_coarse_select", "vsa_coarse_select_tokens", "vsa_tile_permute_pool",
+            "vsa_coarse_select_pooled", "vsa_coarse_select_noalloc",
             "vsa_block_sparse_fwd",
             "vsa_combine", "vsa_untile", "vsa_forward_host_workspace_bytes", "vsa_forward_host",
             "vsa_get_status", "vsa_debug_wait_timeout", "vsa_strerror")
@@ -61,6 +62,8 @@ _sig = {
                                          ctypes.c_size_t, _P]),
     "vsa_coarse_select_tokens": (ctypes.c_int, [_SP, _P, _P, _P, ctypes.c_int, _P, _P, _P, _P,
                                                 ctypes.c_size_t, _P]),
+    "vsa_tile_permute_pool": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "vsa_coarse_select_pooled": (ctypes.c_int, [_SP, ctypes.c_int, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "vsa_coarse_select_noalloc": (ctypes.c_int, [_SP, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P, _P]),
     "vsa_block_sparse_fwd": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P]),
     "vsa_combine": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P]),
@@ -189,6 +192,37 @@ def vsa_coarse_select_tokens(shape, q, k, v, topk, sel_idx, workspace, o_coarse=
                                          _ptr(o_coarse), _ptr(sel_idx), _ptr(coarse_logits),
                                          _ptr(workspace), workspace.numel() * workspace.element_size(),
                                          _stream(stream)), "vsa_coarse_select_tokens")
+
+
+def vsa_tile_permute_pool(shape, q, k, v, q_tiled, k_tiled, v_tiled, workspace, cube_count=None,
+                          stream=None):
+    """Tiles q, k, v and writes their cube means into ``workspace`` in one pass."""
+    B, H, N, d, C = _dims(shape)
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _expect(t, torch.bfloat16, (B, H, N, d), n)
+    for n, t in (("q_tiled", q_tiled), ("k_tiled", k_tiled), ("v_tiled", v_tiled)):
+        _expect(t, torch.bfloat16, (B, H, 64 * C, d), n)
+    if cube_count is not None:
+        _expect(cube_count, torch.int32, (C,), "cube_count")
+    _check(_lib.vsa_tile_permute_pool(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(q_tiled),
+                                      _ptr(k_tiled), _ptr(v_tiled), _ptr(cube_count), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)),
+           "vsa_tile_permute_pool")
+
+
+def vsa_coarse_select_pooled(shape, topk, sel_idx, workspace, o_coarse=None, coarse_logits=None,
+                             stream=None):
+    """The coarse stage from the cube means vsa_tile_permute_pool left in ``workspace``."""
+    B, H, N, d, C = _dims(shape)
+    _expect(sel_idx, torch.int32, (B, H, C, topk), "sel_idx")
+    if o_coarse is not None:
+        _expect(o_coarse, torch.float32, (B, H, C, d), "o_coarse")
+    if coarse_logits is not None:
+        _expect(coarse_logits, torch.float32, (B, H, C, C), "coarse_logits")
+    _check(_lib.vsa_coarse_select_pooled(ctypes.byref(shape), topk, _ptr(o_coarse), _ptr(sel_idx),
+                                         _ptr(coarse_logits), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(stream)),
+           "vsa_coarse_select_pooled")
 
 
 def vsa_coarse_select_noalloc(shape, q_tiled, k_tiled, v_tiled, cube_count, topk, sel_idx,
