@@ -191,6 +191,22 @@ int vsa_block_sparse_fwd(const vsa_shape* shape, const void* q_tiled, const void
                          const int32_t* sel_idx, int topk, void* o_fine_tiled,
                          float* lse, cudaStream_t stream);
 
+/* vsa_block_sparse_fwd whose epilogue writes the FINAL output: each valid row
+ * of O_f goes straight to its token in `out` (token order, as vsa_untile
+ * would put it), and with gates the row is first combined exactly as
+ * vsa_combine does (g_fine * bf16(O_f) + g_coarse * O_c, rounded to bf16).
+ * Same bits as vsa_block_sparse_fwd + vsa_combine + vsa_untile; the pages have
+ * no counterpart: this is the combine and untile steps fused into the fine
+ * kernel, which saves two passes over the output.
+ *   q/k/v_tiled, cube_count, sel_idx, topk, lse   as vsa_block_sparse_fwd
+ *   o_coarse     float32 [B, H, C, d] (may be NULL when the gates are NULL)
+ *   g_fine, g_coarse float32 [B, H, N] in token order, or both NULL
+ *   out          bf16 [B, H, N, d] token order (written) */
+int vsa_block_sparse_fwd_out(const vsa_shape* shape, const void* q_tiled, const void* k_tiled,
+                             const void* v_tiled, const int32_t* cube_count, const int32_t* sel_idx,
+                             int topk, const float* o_coarse, const float* g_fine,
+                             const float* g_coarse, void* out, float* lse, cudaStream_t stream);
+
 /* Optional per-token gated sum of the fine and coarse outputs, in tiled order:
  *   out[r] = g_fine[n] * O_f[r] + g_coarse[n] * O_c[cube of r]
  * where n is the token held by tiled row r.  With g_fine == g_coarse == NULL,
@@ -209,7 +225,7 @@ int vsa_untile(const vsa_shape* shape, const void* x_tiled, void* x, cudaStream_
 
 /* Bytes of device workspace vsa_forward_host needs: two chunk buffers, each
  * holding heads_per_chunk (b, h) planes of the inputs, their tiled copies,
- * the fine and final outputs and the coarse-stage scratch.  heads_per_chunk
+ * the final output and the coarse-stage scratch.  heads_per_chunk
  * 0 means 2; gated is 0 or 1.  Returns 0 for an invalid shape or k. */
 size_t vsa_forward_host_workspace_bytes(const vsa_shape* shape, int topk, int heads_per_chunk,
                                         int gated);

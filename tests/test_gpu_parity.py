@@ -164,6 +164,31 @@ def test_fused_tile_pool_equals_separate_calls(vsa, B, H, d, grid, k):
     assert torch.equal(o_c, bufs.o_c)
 
 
+@pytest.mark.parametrize("name", ["tiny_k2", "wan1.3b_ft_16x28x52", "wan1.3b_480p_21x30x52"])
+def test_fine_with_fused_combine_untile_equals_separate_calls(vsa, name):
+    # the fine kernel writing the final token-order output (gated sum applied
+    # when the workload has gates) gives the same bits as fwd + combine + untile
+    w = wl.WORKLOADS[name]
+    x = wl.make_inputs(w)
+    shape = vsa.make_shape(w.batch, w.heads, w.head_dim, w.grid)
+    q, k, v = (to_dev_bf16(x[n]) for n in ("q", "k", "v"))
+    g_f = torch.from_numpy(x["g_f"]).cuda() if w.gated else None
+    g_c = torch.from_numpy(x["g_c"]).cuda() if w.gated else None
+    want = torch.empty_like(q)
+    bufs = vsa.vsa_forward(shape, q, k, v, w.topk, want, g_f, g_c)
+    got = torch.full_like(q, 3.0)
+    lse = torch.empty(w.batch, w.heads, 64 * w.cubes, dtype=torch.float32, device="cuda")
+    vsa.vsa_block_sparse_fwd_out(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, bufs.sel, w.topk,
+                                 got, bufs.o_c if w.gated else None, g_f, g_c, lse=lse)
+    lse_want = torch.empty_like(lse)
+    vsa.vsa_block_sparse_fwd(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, bufs.sel, w.topk,
+                             bufs.o_f, lse_want)
+    torch.cuda.synchronize()
+    assert vsa.vsa_get_status() == 0
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+    assert torch.equal(lse, lse_want)
+
+
 @pytest.mark.parametrize("grid,k", [((8, 8, 8), 3), ((48, 48, 48), 1700)])
 def test_topk_ties_go_to_lower_index(vsa, grid, k):
     # identical k vectors in every cube -> all coarse logits of a row tie

@@ -99,6 +99,12 @@ def test_null_and_misaligned_pointers_rejected_before_launch(vsa):
     assert tp(ctypes.byref(s), p, p, p, p, p, None, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
     assert tp(ctypes.byref(s), p, p, p, p, p, p, None, p, 16, None) == vsa.VSA_ERR_INVALID_ARG
     assert tp(ctypes.byref(s), p, odd, p, p, p, p, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
+    fo = lib.vsa_block_sparse_fwd_out
+    assert fo(ctypes.byref(s), p, p, p, p, p, 5, None, None, None, p, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert fo(ctypes.byref(s), p, p, p, p, p, 2, None, None, None, None, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert fo(ctypes.byref(s), p, p, p, p, p, 2, None, p, None, p, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert fo(ctypes.byref(s), p, p, p, p, p, 2, None, p, p, p, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert fo(ctypes.byref(s), p, p, p, p, p, 2, None, None, None, odd, None, None) == vsa.VSA_ERR_INVALID_ARG
     cp = lib.vsa_coarse_select_pooled
     assert cp(ctypes.byref(s), 5, None, p, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
     assert cp(ctypes.byref(s), 2, None, None, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
@@ -116,7 +122,7 @@ def test_forward_host_workspace_and_argument_checks(vsa):
     lib = vsa._lib
     s = vsa.make_shape(1, 40, 128, (21, 45, 80))
     C, N, d = 1440, 21 * 45 * 80, 128
-    per_chunk_ungated = (3 * 8 * N * d * 2 + 4 * 8 * 64 * C * d * 2 + 8 * N * d * 2
+    per_chunk_ungated = (3 * 8 * N * d * 2 + 3 * 8 * 64 * C * d * 2 + 8 * N * d * 2
                          + 8 * C * 180 * 4 + 3 * 8 * C * d * 4 + C * 4)
     got = vsa.vsa_forward_host_workspace_bytes(s, 180, 8, gated=False)
     assert per_chunk_ungated * 2 <= got <= per_chunk_ungated * 2 + 2 * 16 * 256

@@ -25,7 +25,8 @@ cudaError_t launch_coarse_only(const Geom&, int, float*, int32_t*, float*, const
                                cudaStream_t);
 cudaError_t launch_block_sparse_fwd(const Geom&, const CUtensorMap&, const CUtensorMap&,
                                     const CUtensorMap&, const int32_t*, const int32_t*, int,
-                                    void*, float*, int*, int, cudaStream_t);
+                                    void*, float*, const float*, const float*, const float*, bool,
+                                    int*, int, cudaStream_t);
 cudaError_t launch_debug_wait(uint64_t, int*, cudaStream_t);
 
 // Device-side status word, one per device that loads the library.
@@ -316,7 +317,40 @@ int vsa_block_sparse_fwd(const vsa_shape* shape, const void* q_tiled, const void
       tiled_map(g, v_tiled, &tv) != VSA_OK)
     return VSA_ERR_CUDA;
   return cuda_rc(launch_block_sparse_fwd(g, tq, tk, tv, cube_count, sel_idx, topk, o_fine_tiled,
-                                         lse, st->status, st->sms, stream));
+                                         lse, nullptr, nullptr, nullptr, false, st->status, st->sms,
+                                         stream));
+}
+
+int vsa_block_sparse_fwd_out(const vsa_shape* shape, const void* q_tiled, const void* k_tiled,
+                             const void* v_tiled, const int32_t* cube_count, const int32_t* sel_idx,
+                             int topk, const float* o_coarse, const float* g_fine,
+                             const float* g_coarse, void* out, float* lse, cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (topk < 1 || topk > g.C) return VSA_ERR_INVALID_ARG;
+  if (!q_tiled || !k_tiled || !v_tiled || !cube_count || !sel_idx || !out)
+    return VSA_ERR_INVALID_ARG;
+  if ((g_fine == nullptr) != (g_coarse == nullptr)) return VSA_ERR_INVALID_ARG;
+  if (g_fine && (!o_coarse || !aligned16(o_coarse) ||
+                 (reinterpret_cast<uintptr_t>(g_fine) & 3u) ||
+                 (reinterpret_cast<uintptr_t>(g_coarse) & 3u)))
+    return VSA_ERR_INVALID_ARG;
+  if (!aligned16(q_tiled) || !aligned16(k_tiled) || !aligned16(v_tiled) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(cube_count) & 3u) ||
+      (reinterpret_cast<uintptr_t>(sel_idx) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return VSA_ERR_INVALID_ARG;
+  DeviceState* st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  if ((rc = get_encoder()) != VSA_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  if (tiled_map(g, q_tiled, &tq) != VSA_OK || tiled_map(g, k_tiled, &tk) != VSA_OK ||
+      tiled_map(g, v_tiled, &tv) != VSA_OK)
+    return VSA_ERR_CUDA;
+  return cuda_rc(launch_block_sparse_fwd(g, tq, tk, tv, cube_count, sel_idx, topk, out, lse,
+                                         g_fine ? o_coarse : nullptr, g_fine, g_coarse, true,
+                                         st->status, st->sms, stream));
 }
 
 int vsa_get_status(cudaStream_t stream) {

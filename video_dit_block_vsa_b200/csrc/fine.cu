@@ -66,6 +66,18 @@ struct Cfg {
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(64, D, false, true);  // P (TMEM), V MN-major
 };
 
+// Where the epilogue writes O / l: the tiled bf16 tensor, or (token_order)
+// the final bf16 output in token order, optionally as the gated sum
+// g_f * bf16(O / l) + g_c * O_c of the combine step.
+struct OutSpec {
+  __nv_bfloat16* out;
+  float* lse;
+  const float* o_coarse;
+  const float* g_fine;
+  const float* g_coarse;
+  int token_order;
+};
+
 struct Shared {
   uint64_t* q_full;
   uint64_t* q_empty;
@@ -335,11 +347,12 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
 }
 
 // ------------------------------------------------------------------ softmax
-template <int D>
+template <int D, bool kTokenOut>
 __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c,
-                           const int32_t* __restrict__ sel, int topk,
-                           __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
+                           const int32_t* __restrict__ sel, int topk, const OutSpec os,
                            int* status) {
+  __nv_bfloat16* __restrict__ out = os.out;
+  float* __restrict__ lse = os.lse;
   using Cf = Cfg<D>;
   constexpr int kOH = D / 2;  // O columns per thread (half a row)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -433,7 +446,19 @@ __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c
       tc_fence_before();
       mbar_arrive(&sh.p_full[c]);
     }
-    // ---- epilogue: O / l -> bf16; pad rows -> 0
+    // ---- epilogue: O / l -> bf16; pad rows -> 0 (tiled) or no write (token order)
+    const bool valid = r < ni;
+    // token-order output: the row's token and gates, ahead of the O load so
+    // they are not live beside its registers
+    long long tok = 0;
+    float wf = 0.f, wc = 0.f;
+    if (kTokenOut && valid) {
+      tok = static_cast<long long>(it.bh) * g.N + slot_token(g, i, r);
+      if (os.g_fine != nullptr) {
+        wf = __ldg(&os.g_fine[tok]);
+        wc = __ldg(&os.g_coarse[tok]);
+      }
+    }
     if (!mbar_wait(&sh.o_full[c], o_phase)) return fail(sh, status);
     o_phase ^= 1u;
     tc_fence_after();
@@ -444,20 +469,45 @@ __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c
       tmem_ld_16x32bx2_x32(tO, ov);
     }
     const float l = l_part + __shfl_xor_sync(0xffffffffu, l_part, 16);
-    const bool valid = r < ni;
     const float inv = 1.0f / l;
-    uint4* orow = reinterpret_cast<uint4*>(
-        out + (static_cast<long long>(it.row0) + i * 64 + r) * D + hh * kOH);
+    if (!kTokenOut) {
+      uint4* orow = reinterpret_cast<uint4*>(
+          out + (static_cast<long long>(it.row0) + i * 64 + r) * D + hh * kOH);
 #pragma unroll
-    for (int q8 = 0; q8 < kOH / 8; ++q8) {
-      uint4 w = make_uint4(0u, 0u, 0u, 0u);
-      if (valid) {
-        w.x = pack2_bf16(__uint_as_float(ov[q8 * 8 + 0]) * inv, __uint_as_float(ov[q8 * 8 + 1]) * inv);
-        w.y = pack2_bf16(__uint_as_float(ov[q8 * 8 + 2]) * inv, __uint_as_float(ov[q8 * 8 + 3]) * inv);
-        w.z = pack2_bf16(__uint_as_float(ov[q8 * 8 + 4]) * inv, __uint_as_float(ov[q8 * 8 + 5]) * inv);
-        w.w = pack2_bf16(__uint_as_float(ov[q8 * 8 + 6]) * inv, __uint_as_float(ov[q8 * 8 + 7]) * inv);
+      for (int q8 = 0; q8 < kOH / 8; ++q8) {
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (valid) {
+          w.x = pack2_bf16(__uint_as_float(ov[q8 * 8 + 0]) * inv, __uint_as_float(ov[q8 * 8 + 1]) * inv);
+          w.y = pack2_bf16(__uint_as_float(ov[q8 * 8 + 2]) * inv, __uint_as_float(ov[q8 * 8 + 3]) * inv);
+          w.z = pack2_bf16(__uint_as_float(ov[q8 * 8 + 4]) * inv, __uint_as_float(ov[q8 * 8 + 5]) * inv);
+          w.w = pack2_bf16(__uint_as_float(ov[q8 * 8 + 6]) * inv, __uint_as_float(ov[q8 * 8 + 7]) * inv);
+        }
+        orow[q8] = w;
       }
-      orow[q8] = w;
+    } else if (valid) {
+      // pad rows have no token and write nothing
+      uint4* orow = reinterpret_cast<uint4*>(out + tok * D + hh * kOH);
+      const bool gated = os.g_fine != nullptr;
+      const float4* oc = reinterpret_cast<const float4*>(
+          os.o_coarse + (static_cast<long long>(it.bh) * g.C + i) * D + hh * kOH);
+#pragma unroll
+      for (int q8 = 0; q8 < kOH / 8; ++q8) {
+        uint32_t f[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          f[e] = pack2_bf16(__uint_as_float(ov[q8 * 8 + 2 * e]) * inv,
+                            __uint_as_float(ov[q8 * 8 + 2 * e + 1]) * inv);
+        if (gated) {  // the combine step's arithmetic on the bf16 fine output
+          const float4 c0 = __ldg(&oc[2 * q8]);
+          const float4 c1 = __ldg(&oc[2 * q8 + 1]);
+          const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            f[e] = pack2_bf16(fmaf(wf, __uint_as_float(f[e] << 16), wc * cv[2 * e]),
+                              fmaf(wf, __uint_as_float(f[e] & 0xFFFF0000u), wc * cv[2 * e + 1]));
+        }
+        orow[q8] = make_uint4(f[0], f[1], f[2], f[3]);
+      }
     }
     if (lse != nullptr && hh == 0)
       lse[static_cast<long long>(it.row0) + i * 64 + r] =
@@ -465,12 +515,11 @@ __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c
   }
 }
 
-template <int D>
+template <int D, bool kTokenOut>
 __global__ void __launch_bounds__(kThreads, 1) fine_fwd_kernel(
     const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
     const __grid_constant__ CUtensorMap tv, Geom g, const int32_t* __restrict__ counts,
-    const int32_t* __restrict__ sel, int topk, __nv_bfloat16* __restrict__ out,
-    float* __restrict__ lse, int* status) {
+    const int32_t* __restrict__ sel, int topk, const OutSpec os, int* status) {
   using Cf = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -521,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_fwd_kernel(
   } else if (warp == kMmaWarp) {
     if (lane == 0) mma_issuer<D>(sh, g, tmem, topk, status);
   } else if (warp >= kSoftmaxWarp0) {
-    softmax_wg<D>(sh, g, tmem, (warp - kSoftmaxWarp0) >> 2, sel, topk, out, lse, status);
+    softmax_wg<D, kTokenOut>(sh, g, tmem, (warp - kSoftmaxWarp0) >> 2, sel, topk, os, status);
   }
   tc_fence_before();
   __syncthreads();
@@ -535,23 +584,28 @@ size_t fine_smem_bytes(int d) { return d == 128 ? Cfg<128>::kSmem : Cfg<64>::kSm
 cudaError_t launch_block_sparse_fwd(const Geom& g, const CUtensorMap& tq, const CUtensorMap& tk,
                                     const CUtensorMap& tv, const int32_t* counts,
                                     const int32_t* sel, int topk, void* out, float* lse,
-                                    int* status, int sms, cudaStream_t s) {
+                                    const float* o_coarse, const float* g_fine,
+                                    const float* g_coarse, bool token_order, int* status, int sms,
+                                    cudaStream_t s) {
   const long long items = static_cast<long long>(g.B) * g.H * ((g.C + 1) / 2);
   const int grid = static_cast<int>(items < sms ? items : sms);
   const size_t smem = fine_smem_bytes(g.d);
+  const OutSpec os{static_cast<__nv_bfloat16*>(out), lse, o_coarse, g_fine, g_coarse,
+                   token_order ? 1 : 0};
   cudaError_t err;
-  static unsigned long long limit_set[2] = {0, 0};
-  if (g.d == 128) {
-    err = smem_limit_once(fine_fwd_kernel<128>, static_cast<int>(smem), &limit_set[0]);
-    if (err != cudaSuccess) return err;
-    fine_fwd_kernel<128><<<grid, kThreads, smem, s>>>(tq, tk, tv, g, counts, sel, topk,
-                                                       static_cast<__nv_bfloat16*>(out), lse, status);
-  } else {
-    err = smem_limit_once(fine_fwd_kernel<64>, static_cast<int>(smem), &limit_set[1]);
-    if (err != cudaSuccess) return err;
-    fine_fwd_kernel<64><<<grid, kThreads, smem, s>>>(tq, tk, tv, g, counts, sel, topk,
-                                                      static_cast<__nv_bfloat16*>(out), lse, status);
-  }
+  // one kernel per head dim and output form; each raises its smem limit once
+  static unsigned long long limit_set[4] = {0, 0, 0, 0};
+  auto run = [&](auto kernel, int which) -> cudaError_t {
+    cudaError_t e = smem_limit_once(kernel, static_cast<int>(smem), &limit_set[which]);
+    if (e != cudaSuccess) return e;
+    kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, g, counts, sel, topk, os, status);
+    return cudaSuccess;
+  };
+  if (g.d == 128)
+    err = token_order ? run(fine_fwd_kernel<128, true>, 0) : run(fine_fwd_kernel<128, false>, 1);
+  else
+    err = token_order ? run(fine_fwd_kernel<64, true>, 2) : run(fine_fwd_kernel<64, false>, 3);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 

@@ -3,9 +3,9 @@
 // computes on the caller's stream, the next chunk's q, k, v (and gates) are
 // copied in on one internal stream and the previous chunk's output is copied
 // out on another, so PCIe transfers in both directions overlap the kernels.
-// Every stage runs through the same entry points as the device-buffer path
-// (tiling and pooling in one pass, then the coarse stage, fine stage, combine
-// and untile).
+// Every stage runs through the library's own entry points: tiling and pooling
+// in one pass, the coarse stage, and the fine stage writing the final output
+// (gated combine and untile in its epilogue).
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -50,7 +50,7 @@ size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Byte offsets of one chunk buffer inside the workspace.
 struct ChunkLayout {
-  size_t x[3], g[2], xt[3], of, out, oc, sel, pool, counts, total;
+  size_t x[3], g[2], xt[3], out, oc, sel, pool, counts, total;
 };
 
 ChunkLayout chunk_layout(int C, long long N, int d, int topk, int hc, bool gated) {
@@ -64,7 +64,6 @@ ChunkLayout chunk_layout(int C, long long N, int d, int topk, int hc, bool gated
     if (gated) off += round256(static_cast<size_t>(hc) * N * 4);
   }
   for (int i = 0; i < 3; ++i) { L.xt[i] = off; off += round256(til); }
-  L.of = off; off += round256(til);
   L.out = off; off += round256(tok);
   L.oc = off; if (gated) off += round256(static_cast<size_t>(hc) * C * d * 4);
   L.sel = off; off += round256(static_cast<size_t>(hc) * C * topk * 4);
@@ -189,13 +188,11 @@ int vsa_forward_host(const vsa_shape* shape, int topk, const void* q, const void
                                     base + L.pool, pool_bytes, stream)) != VSA_OK ||
         (rc = vsa_coarse_select_pooled(&sub, topk, oc, sel, nullptr, base + L.pool, pool_bytes,
                                        stream)) != VSA_OK ||
-        (rc = vsa_block_sparse_fwd(&sub, base + L.xt[0], base + L.xt[1], base + L.xt[2], counts,
-                                   sel, topk, base + L.of, nullptr, stream)) != VSA_OK ||
-        (rc = vsa_combine(&sub, base + L.of, oc,
-                          gated ? reinterpret_cast<const float*>(base + L.g[0]) : nullptr,
-                          gated ? reinterpret_cast<const float*>(base + L.g[1]) : nullptr,
-                          base + L.of, stream)) != VSA_OK ||
-        (rc = vsa_untile(&sub, base + L.of, base + L.out, stream)) != VSA_OK)
+        (rc = vsa_block_sparse_fwd_out(
+             &sub, base + L.xt[0], base + L.xt[1], base + L.xt[2], counts, sel, topk, oc,
+             gated ? reinterpret_cast<const float*>(base + L.g[0]) : nullptr,
+             gated ? reinterpret_cast<const float*>(base + L.g[1]) : nullptr, base + L.out,
+             nullptr, stream)) != VSA_OK)
       return finish(rc);
     if (cudaEventRecord(ev_done[b], stream) != cudaSuccess) return finish(VSA_ERR_CUDA);
     // output

@@ -34,7 +34,7 @@ VSA_ERR_TOO_LARGE = 6
 EXPORTED = ("vsa_num_cubes", "vsa_topk_from_ratio", "vsa_workspace_bytes", "vsa_tile_permute",
             "vsa_coarse_select", "vsa_coarse_select_tokens", "vsa_tile_permute_pool",
             "vsa_coarse_select_pooled", "vsa_coarse_select_noalloc",
-            "vsa_block_sparse_fwd",
+            "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_out",
             "vsa_combine", "vsa_untile", "vsa_forward_host_workspace_bytes", "vsa_forward_host",
             "vsa_get_status", "vsa_debug_wait_timeout", "vsa_strerror")
 
@@ -66,6 +66,8 @@ _sig = {
     "vsa_coarse_select_pooled": (ctypes.c_int, [_SP, ctypes.c_int, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "vsa_coarse_select_noalloc": (ctypes.c_int, [_SP, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P, _P]),
     "vsa_block_sparse_fwd": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P]),
+    "vsa_block_sparse_fwd_out": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P,
+                                                _P, _P, _P]),
     "vsa_combine": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P]),
     "vsa_untile": (ctypes.c_int, [_SP, _P, _P, _P]),
     "vsa_forward_host_workspace_bytes": (ctypes.c_size_t, [_SP, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
@@ -259,6 +261,27 @@ def vsa_block_sparse_fwd(shape, q_tiled, k_tiled, v_tiled, cube_count, sel_idx, 
                                      _ptr(v_tiled), _ptr(cube_count), _ptr(sel_idx), topk,
                                      _ptr(o_fine_tiled), _ptr(lse), _stream(stream)),
            "vsa_block_sparse_fwd")
+
+
+def vsa_block_sparse_fwd_out(shape, q_tiled, k_tiled, v_tiled, cube_count, sel_idx, topk, out,
+                             o_coarse=None, g_fine=None, g_coarse=None, lse=None, stream=None):
+    """Fine stage writing the final token-order output (gated combine and untile fused)."""
+    B, H, N, d, C = _dims(shape)
+    for n, t in (("q_tiled", q_tiled), ("k_tiled", k_tiled), ("v_tiled", v_tiled)):
+        _expect(t, torch.bfloat16, (B, H, 64 * C, d), n)
+    _expect(cube_count, torch.int32, (C,), "cube_count")
+    _expect(sel_idx, torch.int32, (B, H, C, topk), "sel_idx")
+    _expect(out, torch.bfloat16, (B, H, N, d), "out")
+    if g_fine is not None:
+        _expect(g_fine, torch.float32, (B, H, N), "g_fine")
+        _expect(g_coarse, torch.float32, (B, H, N), "g_coarse")
+        _expect(o_coarse, torch.float32, (B, H, C, d), "o_coarse")
+    if lse is not None:
+        _expect(lse, torch.float32, (B, H, 64 * C), "lse")
+    _check(_lib.vsa_block_sparse_fwd_out(ctypes.byref(shape), _ptr(q_tiled), _ptr(k_tiled),
+                                         _ptr(v_tiled), _ptr(cube_count), _ptr(sel_idx), topk,
+                                         _ptr(o_coarse), _ptr(g_fine), _ptr(g_coarse), _ptr(out),
+                                         _ptr(lse), _stream(stream)), "vsa_block_sparse_fwd_out")
 
 
 def vsa_combine(shape, o_fine_tiled, out_tiled, o_coarse=None, g_fine=None, g_coarse=None,
