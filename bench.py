@@ -365,7 +365,7 @@ def run_gpu(args, w):
             "peak_kind": f"{TMA_INGEST_GBS_PER_SM} GB/s per SM (measured) x {sms} SMs"}
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_sustained"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"], "traffic": traffic,
-                "kernel": "vsa_block_sparse_fwd", "peak_kind": f"bf16 sustained ({peaks['source']})",
+                "kernel": "vsa_block_sparse_fwd_out (fine attention; combine and untile in its epilogue)", "peak_kind": f"bf16 sustained ({peaks['source']})",
                 "peak_burst": peaks["bf16"], "frac_of_burst": achieved / peaks["bf16"],
                 "issued_tflops": fine_issued / (fine_ms * 1e-3) / 1e12, "feed": feed}
 
@@ -423,7 +423,7 @@ HOST_CHUNK_HEADS = 2
 
 # Revision tag of the fine kernel; ncu traffic figures are only reported for
 # the revision they were captured on.
-KERNEL_REV = "fine-v3.2"
+KERNEL_REV = "fine-v3.2-out"
 
 
 def main():
