@@ -28,3 +28,30 @@ def test_reference_arm_prints_one_contract_line():
     assert line["config"]["workload"] == "tiny_k2"
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_flop_accounting_counts_valid_token_pairs():
+    # effective FLOPs = 4 d x (number of (query token, selected key token) pairs
+    # over valid tokens); issued FLOPs count every 64x64 tile in full
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import bench
+    from oracle import vsa_oracle as vo
+    from video_dit_block_vsa_b200 import workloads as wl
+    w = wl.Workload("t", 2, 3, 16, (5, 6, 7), 3, 9, 0.5, False)
+    counts = bench.cube_counts(w.grid)
+    assert np.array_equal(counts, vo.cube_permutation(w.grid)[1])
+    rng = np.random.default_rng(0)
+    C = counts.shape[0]
+    sel = np.stack([np.sort(rng.choice(C, w.topk, replace=False)) for _ in range(2 * 3 * C)])
+    sel = sel.reshape(2, 3, C, w.topk)
+    eff, issued, coarse = bench.flop_counts(w, counts, sel)
+    pairs = 0
+    for b in range(2):
+        for h in range(3):
+            for i in range(C):
+                for j in sel[b, h, i]:
+                    pairs += int(counts[i]) * int(counts[j])
+    assert eff == 4.0 * w.head_dim * pairs
+    assert issued == 4.0 * w.head_dim * 2 * 3 * C * w.topk * 64 * 64
+    assert coarse == 4.0 * w.head_dim * 2 * 3 * C * C
