@@ -59,6 +59,40 @@ def attention_backward(Q, K, V, dO, scale):
     return dQ, dK, dV
 
 
+def attention_backward_from_lse(Q, K, V, O, dO, lse, scale):
+    """The same gradients written the way a kernel that saved the forward's
+    natural-log log-sum-exp computes them: P = exp(S - lse), D = rowsum(dO * O),
+    with O the forward output (no second softmax normalisation)."""
+    P = np.exp((Q @ K.T) * scale - lse[:, None])
+    D = np.sum(dO * O, axis=1, keepdims=True)
+    dV = P.T @ dO
+    dS = P * (dO @ V.T - D)
+    return (dS @ K) * scale, (dS.T @ Q) * scale, dV
+
+
+def select_transpose(sel, C):
+    """For every key cube, the query cubes that selected it, ascending.
+
+    sel: [..., C, k] selections (each row ascending, no repeats).  Returns
+    (offsets [..., C + 1], queries [..., C * k]): the query cubes of key cube j
+    are queries[..., offsets[j]:offsets[j + 1]].  The dK/dV side of a backward
+    walks these lists.
+    """
+    lead = sel.shape[:-2]
+    k = sel.shape[-1]
+    flat = sel.reshape(-1, C, k)
+    offs = np.zeros((flat.shape[0], C + 1), dtype=np.int64)
+    qs = np.zeros((flat.shape[0], C * k), dtype=np.int64)
+    for p in range(flat.shape[0]):
+        lists = [[] for _ in range(C)]
+        for i in range(C):  # ascending query cubes keep each list ascending
+            for j in flat[p, i]:
+                lists[int(j)].append(i)
+        offs[p, 1:] = np.cumsum([len(l) for l in lists])
+        qs[p] = np.concatenate([np.asarray(l, dtype=np.int64) for l in lists])
+    return offs.reshape(lead + (C + 1,)), qs.reshape(lead + (C * k,))
+
+
 def block_sparse_attention_backward(qt, kt, vt, counts, sel, dof_t):
     """Gradients of the fine stage w.r.t. the tiled q, k, v.
 
@@ -162,5 +196,6 @@ def vsa_backward(q, k, v, grid, topk, dout, g_f=None, g_c=None, cube=CUBE):
                 dv=untile(dv_t, grid, cube), dg_f=dgf, dg_c=dgc, sel=sel)
 
 
-__all__ = ["attention_backward", "block_sparse_attention_backward", "coarse_attention_backward",
-           "pool_backward", "combine_backward", "vsa_backward"]
+__all__ = ["attention_backward", "attention_backward_from_lse", "select_transpose",
+           "block_sparse_attention_backward", "coarse_attention_backward", "pool_backward",
+           "combine_backward", "vsa_backward"]

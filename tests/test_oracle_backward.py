@@ -132,3 +132,38 @@ def test_pool_backward_spreads_the_mean_gradient_over_valid_rows():
         block = dx[0, 0, 64 * c:64 * (c + 1)]
         np.testing.assert_allclose(block[:n].sum(axis=0), dxb[0, 0, c], atol=1e-12)
         assert np.all(block[n:] == 0)
+
+
+def test_backward_from_saved_lse_equals_recomputed_softmax():
+    # the recipe a kernel with the forward's LSE follows gives the same gradients
+    grid = (5, 6, 7)
+    q, k, v, dout, _, _ = inputs(grid, B=1, H=1, d=8, seed=7, gated=False)
+    q_t, counts = vo.tile_permute(q, grid)
+    k_t, _ = vo.tile_permute(k, grid)
+    v_t, _ = vo.tile_permute(v, grid)
+    do_t, _ = vo.tile_permute(dout, grid)
+    C = counts.shape[0]
+    sel = np.stack([np.arange(C)[::2][:3]] * C).reshape(1, 1, C, 3)
+    O, lse = vo.block_sparse_attention(q_t, k_t, v_t, counts, sel)
+    scale = 1.0 / math.sqrt(q.shape[-1])
+    for i in range(C):
+        rows = slice(64 * i, 64 * i + int(counts[i]))
+        keys = np.concatenate([np.arange(64 * j, 64 * j + int(counts[j])) for j in sel[0, 0, i]])
+        a = vb.attention_backward(q_t[0, 0, rows], k_t[0, 0, keys], v_t[0, 0, keys], do_t[0, 0, rows], scale)
+        b = vb.attention_backward_from_lse(q_t[0, 0, rows], k_t[0, 0, keys], v_t[0, 0, keys],
+                                           O[0, 0, rows], do_t[0, 0, rows], lse[0, 0, rows], scale)
+        for x, y in zip(a, b):
+            np.testing.assert_allclose(x, y, rtol=0, atol=1e-12)
+
+
+def test_select_transpose_is_the_inverse_incidence():
+    rng = np.random.default_rng(4)
+    C, k = 11, 4
+    sel = np.stack([np.sort(rng.choice(C, k, replace=False)) for _ in range(2 * C)]).reshape(2, C, k)
+    offs, qs = vb.select_transpose(sel, C)
+    for p in range(2):
+        assert offs[p, 0] == 0 and offs[p, -1] == C * k
+        for j in range(C):
+            got = qs[p, offs[p, j]:offs[p, j + 1]]
+            want = [i for i in range(C) if j in sel[p, i]]  # brute force
+            assert list(got) == want
