@@ -254,6 +254,21 @@ int vsa_forward_host(const vsa_shape* shape, int topk, const void* q, const void
                      void* workspace, size_t workspace_bytes, int heads_per_chunk,
                      cudaStream_t stream);
 
+/* Transpose of a selection, for the key-stationary side of a backward pass:
+ * for every key cube j of every (b, h), the query cubes i with j in
+ * sel_idx[b, h, i, :], in ascending order, as a CSR list.  The pages have no
+ * counterpart (they describe no backward kernel); it is a building block.
+ *   sel_idx      int32 [B, H, C, k], rows ascending without repeats (as
+ *                vsa_coarse_select writes them); an index outside [0, C) is
+ *                recorded as VSA_ERR_BAD_INDEX and left out
+ *   key_offsets  int32 [B, H, C + 1] (written): key cube j's list is
+ *                query_lists[b, h, key_offsets[b, h, j] .. key_offsets[b, h, j + 1])
+ *   query_lists  int32 [B, H, C * k] (written)
+ *   workspace    device scratch of at least B*H*C*k*4 bytes, 256-byte aligned */
+int vsa_select_transpose(const vsa_shape* shape, const int32_t* sel_idx, int topk,
+                         int32_t* key_offsets, int32_t* query_lists, void* workspace,
+                         size_t workspace_bytes, cudaStream_t stream);
+
 /* Synchronises `stream`, then returns and clears the status word of the
  * current device: VSA_OK, VSA_ERR_TIMEOUT or VSA_ERR_BAD_INDEX recorded by a
  * kernel since the last call, or VSA_ERR_CUDA if the synchronisation failed. */

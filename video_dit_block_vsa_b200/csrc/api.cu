@@ -28,6 +28,8 @@ cudaError_t launch_block_sparse_fwd(const Geom&, const CUtensorMap&, const CUten
                                     void*, float*, const float*, const float*, const float*, bool,
                                     int*, int, cudaStream_t);
 cudaError_t launch_debug_wait(uint64_t, int*, cudaStream_t);
+cudaError_t launch_select_transpose(int, int, int, const int32_t*, int32_t*, int32_t*, int32_t*,
+                                    int*, cudaStream_t);
 
 // Device-side status word, one per device that loads the library.
 __device__ int g_status;
@@ -351,6 +353,26 @@ int vsa_block_sparse_fwd_out(const vsa_shape* shape, const void* q_tiled, const 
   return cuda_rc(launch_block_sparse_fwd(g, tq, tk, tv, cube_count, sel_idx, topk, out, lse,
                                          g_fine ? o_coarse : nullptr, g_fine, g_coarse, true,
                                          st->status, st->sms, stream));
+}
+
+int vsa_select_transpose(const vsa_shape* shape, const int32_t* sel_idx, int topk,
+                         int32_t* key_offsets, int32_t* query_lists, void* workspace,
+                         size_t workspace_bytes, cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (topk < 1 || topk > g.C) return VSA_ERR_INVALID_ARG;
+  if (!sel_idx || !key_offsets || !query_lists || !workspace) return VSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(sel_idx) & 3u) || (reinterpret_cast<uintptr_t>(key_offsets) & 3u) ||
+      (reinterpret_cast<uintptr_t>(query_lists) & 3u) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return VSA_ERR_INVALID_ARG;
+  const long long pairs = static_cast<long long>(g.B) * g.H * g.C * topk;
+  if (static_cast<long long>(g.C) * topk >= (1ll << 31)) return VSA_ERR_UNSUPPORTED;
+  if (workspace_bytes < static_cast<size_t>(pairs) * sizeof(int32_t)) return VSA_ERR_INVALID_ARG;
+  DeviceState* st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  return cuda_rc(launch_select_transpose(g.B * g.H, g.C, topk, sel_idx, key_offsets, query_lists,
+                                         static_cast<int32_t*>(workspace), st->status, stream));
 }
 
 int vsa_get_status(cudaStream_t stream) {

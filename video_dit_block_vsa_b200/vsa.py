@@ -36,7 +36,7 @@ EXPORTED = ("vsa_num_cubes", "vsa_topk_from_ratio", "vsa_workspace_bytes", "vsa_
             "vsa_coarse_select_pooled", "vsa_coarse_select_noalloc",
             "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_out",
             "vsa_combine", "vsa_untile", "vsa_forward_host_workspace_bytes", "vsa_forward_host",
-            "vsa_get_status", "vsa_debug_wait_timeout", "vsa_strerror")
+            "vsa_select_transpose", "vsa_get_status", "vsa_debug_wait_timeout", "vsa_strerror")
 
 
 class VsaShape(ctypes.Structure):
@@ -73,6 +73,7 @@ _sig = {
     "vsa_forward_host_workspace_bytes": (ctypes.c_size_t, [_SP, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "vsa_forward_host": (ctypes.c_int, [_SP, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                         ctypes.c_int, _P]),
+    "vsa_select_transpose": (ctypes.c_int, [_SP, _P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
     "vsa_get_status": (ctypes.c_int, [_P]),
     "vsa_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
     "vsa_strerror": (ctypes.c_char_p, [ctypes.c_int]),
@@ -340,6 +341,18 @@ def vsa_forward_host(shape, topk, q, k, v, out, workspace, g_fine=None, g_coarse
                                  _ptr(g_coarse), _ptr(out), _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), heads_per_chunk,
                                  _stream(stream)), "vsa_forward_host")
+
+
+def vsa_select_transpose(shape, sel_idx, topk, key_offsets, query_lists, workspace, stream=None):
+    """For every key cube, the query cubes that selected it (ascending), as CSR."""
+    B, H, N, d, C = _dims(shape)
+    _expect(sel_idx, torch.int32, (B, H, C, topk), "sel_idx")
+    _expect(key_offsets, torch.int32, (B, H, C + 1), "key_offsets")
+    _expect(query_lists, torch.int32, (B, H, C * topk), "query_lists")
+    _check(_lib.vsa_select_transpose(ctypes.byref(shape), _ptr(sel_idx), topk, _ptr(key_offsets),
+                                     _ptr(query_lists), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream)),
+           "vsa_select_transpose")
 
 
 def vsa_get_status(stream=None) -> int:
