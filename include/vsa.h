@@ -269,6 +269,23 @@ int vsa_select_transpose(const vsa_shape* shape, const int32_t* sel_idx, int top
                          int32_t* key_offsets, int32_t* query_lists, void* workspace,
                          size_t workspace_bytes, cudaStream_t stream);
 
+/* First pass of a backward: the gradient of the gated combine, in the layouts
+ * the attention backward reads, in one pass over dout (selection held fixed;
+ * the pages describe no backward, this follows from differentiating the
+ * forward).  With out = g_f O_f + g_c O_c[cube] (or out = O_f ungated):
+ *   do_fine_tiled bf16 [B, H, 64*C, d] (written): bf16(g_f * dout), tiled, pad rows 0
+ *   delta         float32 [B, H, 64*C] (written): sum over d of do_fine * O_f, pad rows 0
+ *   do_coarse     float32 [B, H, C, d] (written, gated only): sum over the cube's
+ *                 valid tokens of g_c * dout
+ *   dg_fine, dg_coarse float32 [B, H, N] (written, gated only): <dout, O_f>, <dout, O_c[cube]>
+ * Inputs: dout bf16 [B, H, N, d] token order; o_fine_tiled bf16 [B, H, 64*C, d]
+ * (the forward's O_f); o_coarse float32 [B, H, C, d] and the gates as in
+ * vsa_combine, all three NULL when ungated. */
+int vsa_backward_prep(const vsa_shape* shape, const void* dout, const void* o_fine_tiled,
+                      const float* o_coarse, const float* g_fine, const float* g_coarse,
+                      void* do_fine_tiled, float* delta, float* do_coarse, float* dg_fine,
+                      float* dg_coarse, cudaStream_t stream);
+
 /* Synchronises `stream`, then returns and clears the status word of the
  * current device: VSA_OK, VSA_ERR_TIMEOUT or VSA_ERR_BAD_INDEX recorded by a
  * kernel since the last call, or VSA_ERR_CUDA if the synchronisation failed. */

@@ -110,6 +110,11 @@ def test_null_and_misaligned_pointers_rejected_before_launch(vsa):
     assert st(ctypes.byref(s), p, 2, None, p, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
     assert st(ctypes.byref(s), p, 2, p, p, p, 16, None) == vsa.VSA_ERR_INVALID_ARG
     assert st(ctypes.byref(s), p, 2, p, p, ctypes.c_void_p(0x100010), 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
+    bp = lib.vsa_backward_prep
+    assert bp(ctypes.byref(s), None, p, None, None, None, p, p, None, None, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert bp(ctypes.byref(s), p, p, None, p, None, p, p, None, None, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert bp(ctypes.byref(s), p, p, None, p, p, p, p, p, p, p, None) == vsa.VSA_ERR_INVALID_ARG
+    assert bp(ctypes.byref(s), odd, p, None, None, None, p, p, None, None, None, None) == vsa.VSA_ERR_INVALID_ARG
     cp = lib.vsa_coarse_select_pooled
     assert cp(ctypes.byref(s), 5, None, p, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
     assert cp(ctypes.byref(s), 2, None, None, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG

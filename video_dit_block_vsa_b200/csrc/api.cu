@@ -30,6 +30,8 @@ cudaError_t launch_block_sparse_fwd(const Geom&, const CUtensorMap&, const CUten
 cudaError_t launch_debug_wait(uint64_t, int*, cudaStream_t);
 cudaError_t launch_select_transpose(int, int, int, const int32_t*, int32_t*, int32_t*, int32_t*,
                                     int*, cudaStream_t);
+cudaError_t launch_backward_prep(const Geom&, const void*, const void*, const float*, const float*,
+                                 const float*, void*, float*, float*, float*, float*, cudaStream_t);
 
 // Device-side status word, one per device that loads the library.
 __device__ int g_status;
@@ -373,6 +375,31 @@ int vsa_select_transpose(const vsa_shape* shape, const int32_t* sel_idx, int top
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_select_transpose(g.B * g.H, g.C, topk, sel_idx, key_offsets, query_lists,
                                          static_cast<int32_t*>(workspace), st->status, stream));
+}
+
+int vsa_backward_prep(const vsa_shape* shape, const void* dout, const void* o_fine_tiled,
+                      const float* o_coarse, const float* g_fine, const float* g_coarse,
+                      void* do_fine_tiled, float* delta, float* do_coarse, float* dg_fine,
+                      float* dg_coarse, cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (!dout || !o_fine_tiled || !do_fine_tiled || !delta) return VSA_ERR_INVALID_ARG;
+  if ((g_fine == nullptr) != (g_coarse == nullptr)) return VSA_ERR_INVALID_ARG;
+  const bool gated = g_fine != nullptr;
+  if (gated && (!o_coarse || !do_coarse || !dg_fine || !dg_coarse)) return VSA_ERR_INVALID_ARG;
+  auto a4 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; };
+  if (!aligned16(dout) || !aligned16(o_fine_tiled) || !aligned16(do_fine_tiled) || !a4(delta))
+    return VSA_ERR_INVALID_ARG;
+  if (gated && (!aligned16(o_coarse) || !aligned16(do_coarse) || !a4(g_fine) || !a4(g_coarse) ||
+                !a4(dg_fine) || !a4(dg_coarse)))
+    return VSA_ERR_INVALID_ARG;
+  DeviceState* st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  return cuda_rc(launch_backward_prep(g, dout, o_fine_tiled, gated ? o_coarse : nullptr,
+                                      g_fine, g_coarse, do_fine_tiled, delta,
+                                      gated ? do_coarse : nullptr, gated ? dg_fine : nullptr,
+                                      gated ? dg_coarse : nullptr, stream));
 }
 
 int vsa_get_status(cudaStream_t stream) {

@@ -36,7 +36,8 @@ EXPORTED = ("vsa_num_cubes", "vsa_topk_from_ratio", "vsa_workspace_bytes", "vsa_
             "vsa_coarse_select_pooled", "vsa_coarse_select_noalloc",
             "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_out",
             "vsa_combine", "vsa_untile", "vsa_forward_host_workspace_bytes", "vsa_forward_host",
-            "vsa_select_transpose", "vsa_get_status", "vsa_debug_wait_timeout", "vsa_strerror")
+            "vsa_select_transpose", "vsa_backward_prep", "vsa_get_status", "vsa_debug_wait_timeout",
+            "vsa_strerror")
 
 
 class VsaShape(ctypes.Structure):
@@ -74,6 +75,7 @@ _sig = {
     "vsa_forward_host": (ctypes.c_int, [_SP, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                         ctypes.c_int, _P]),
     "vsa_select_transpose": (ctypes.c_int, [_SP, _P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
+    "vsa_backward_prep": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "vsa_get_status": (ctypes.c_int, [_P]),
     "vsa_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
     "vsa_strerror": (ctypes.c_char_p, [ctypes.c_int]),
@@ -353,6 +355,25 @@ def vsa_select_transpose(shape, sel_idx, topk, key_offsets, query_lists, workspa
                                      _ptr(query_lists), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream(stream)),
            "vsa_select_transpose")
+
+
+def vsa_backward_prep(shape, dout, o_fine_tiled, do_fine_tiled, delta, o_coarse=None, g_fine=None,
+                      g_coarse=None, do_coarse=None, dg_fine=None, dg_coarse=None, stream=None):
+    """Gradient of the gated combine, ready for the attention backward (see vsa.h)."""
+    B, H, N, d, C = _dims(shape)
+    _expect(dout, torch.bfloat16, (B, H, N, d), "dout")
+    _expect(o_fine_tiled, torch.bfloat16, (B, H, 64 * C, d), "o_fine_tiled")
+    _expect(do_fine_tiled, torch.bfloat16, (B, H, 64 * C, d), "do_fine_tiled")
+    _expect(delta, torch.float32, (B, H, 64 * C), "delta")
+    if g_fine is not None:
+        for n, t, shp in (("o_coarse", o_coarse, (B, H, C, d)), ("do_coarse", do_coarse, (B, H, C, d)),
+                          ("g_fine", g_fine, (B, H, N)), ("g_coarse", g_coarse, (B, H, N)),
+                          ("dg_fine", dg_fine, (B, H, N)), ("dg_coarse", dg_coarse, (B, H, N))):
+            _expect(t, torch.float32, shp, n)
+    _check(_lib.vsa_backward_prep(ctypes.byref(shape), _ptr(dout), _ptr(o_fine_tiled), _ptr(o_coarse),
+                                  _ptr(g_fine), _ptr(g_coarse), _ptr(do_fine_tiled), _ptr(delta),
+                                  _ptr(do_coarse), _ptr(dg_fine), _ptr(dg_coarse), _stream(stream)),
+           "vsa_backward_prep")
 
 
 def vsa_get_status(stream=None) -> int:
