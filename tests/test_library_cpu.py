@@ -165,3 +165,40 @@ def test_forward_host_workspace_and_argument_checks(vsa):
     assert call(*a) == vsa.VSA_ERR_INVALID_ARG
     a = list(ok_args); a[9] = -2                         # negative chunk
     assert call(*a) == vsa.VSA_ERR_INVALID_ARG
+
+
+def test_header_compiles_as_c_and_a_c_program_links_the_library(vsa, tmp_path):
+    # the boundary is a C ABI: a plain C translation unit includes the header,
+    # links libvsa.so and calls the host-only entry points (no GPU needed)
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    cuda_inc = "/usr/local/cuda/include"
+    if gcc is None or not os.path.exists(os.path.join(cuda_inc, "cuda_runtime_api.h")):
+        pytest.skip("gcc or the CUDA headers are not available")
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "vsa.h"
+int main(void) {
+  vsa_shape s = {1, 40, 128, 21, 45, 80, 4, 4, 4};
+  int c = 0, k = 0;
+  if (vsa_num_cubes(&s, &c) != VSA_OK || c != 1440) return 1;
+  if (vsa_topk_from_ratio(c, 0.125f, &k) != VSA_OK || k != 180) return 2;
+  if (vsa_workspace_bytes(&s, k) != (size_t)3 * 40 * 1440 * 128 * 4) return 3;
+  if (strcmp(vsa_strerror(VSA_OK), "ok") != 0) return 4;
+  if (vsa_tile_permute(&s, NULL, NULL, NULL, 0) != VSA_ERR_INVALID_ARG) return 5;
+  printf("c abi ok\n");
+  return 0;
+}
+''')
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(vsa._LIB_PATH)
+    res = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-x", "c", str(src), "-o", str(exe),
+                          f"-I{os.path.join(ROOT, 'include')}", f"-I{cuda_inc}", f"-L{libdir}",
+                          "-lvsa", f"-Wl,-rpath,{libdir}"], capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, (run.returncode, run.stderr)
+    assert "c abi ok" in run.stdout
