@@ -286,6 +286,24 @@ int vsa_backward_prep(const vsa_shape* shape, const void* dout, const void* o_fi
                       void* do_fine_tiled, float* delta, float* do_coarse, float* dg_fine,
                       float* dg_coarse, cudaStream_t stream);
 
+/* Backward of the coarse attention O_c = softmax(qbar kbar^T / sqrt(d)) vbar
+ * (the coarse stage of vsa_coarse_select; the pages describe no backward, this
+ * differentiates that forward exactly, in float32):
+ *   pooled    float32 [3, B, H, C, d]: qbar, kbar, vbar, the layout
+ *             vsa_tile_permute_pool / vsa_coarse_select leave at the start of
+ *             their workspace (read)
+ *   o_coarse  float32 [B, H, C, d]: the forward's O_c (read)
+ *   do_coarse float32 [B, H, C, d]: gradient of O_c, e.g. from vsa_backward_prep (read)
+ *   d_pooled  float32 [3, B, H, C, d]: dqbar, dkbar, dvbar (written)
+ *   workspace device scratch of at least 3*B*H*C*4 bytes, 256-byte aligned
+ *             (per query cube: the row max, 1/z and <do_coarse, o_coarse>)
+ * All float pointers 16-byte aligned; B*H at most 65535.  No C x C matrix is
+ * stored: a row pass gives dqbar and the softmax statistics, a column pass
+ * recomputes P from them for dkbar and dvbar. */
+int vsa_coarse_backward(const vsa_shape* shape, const float* pooled, const float* o_coarse,
+                        const float* do_coarse, float* d_pooled, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream);
+
 /* Synchronises `stream`, then returns and clears the status word of the
  * current device: VSA_OK, VSA_ERR_TIMEOUT or VSA_ERR_BAD_INDEX recorded by a
  * kernel since the last call, or VSA_ERR_CUDA if the synchronisation failed. */

@@ -1,5 +1,6 @@
 """vsa_backward_prep (gradient of the gated combine, first pass of a backward)
-against the oracle's combine_backward on the same bf16 inputs: the fine-branch
+against the oracle's combine_backward on the same bf16 inputs (the forward's
+O_f and O_c taken from the oracle): the fine-branch
 gradient within bf16 rounding, the float32 row sums, gate gradients and the
 coarse-branch gradient within float32 accumulation, pad rows exactly zero."""
 
@@ -33,28 +34,36 @@ def test_backward_prep_matches_combine_backward(vsa, w):
     x = wl.make_inputs(w)
     shape = vsa.make_shape(w.batch, w.heads, w.head_dim, w.grid)
     B, H, N, d, C = w.batch, w.heads, w.tokens, w.head_dim, w.cubes
-    q, k, v = (to_dev_bf16(x[n]) for n in ("q", "k", "v"))
+    # the forward's O_f and O_c come from the oracle (rounded to the types the
+    # kernel reads), so no input of the check is produced by the CUDA path
+    f64 = lambda n: vo.bf16_bits_to_f64(x[n])
+    q_t, counts = vo.tile_permute(f64("q"), w.grid)
+    k_t, _ = vo.tile_permute(f64("k"), w.grid)
+    v_t, _ = vo.tile_permute(f64("v"), w.grid)
+    S_c, oc_ref = vo.coarse_attention(vo.pool(q_t, counts), vo.pool(k_t, counts), vo.pool(v_t, counts))
+    of_ref, _ = vo.block_sparse_attention(q_t, k_t, v_t, counts, vo.topk_select(S_c, w.topk))
+    of_bits = wl.f32_to_bf16_bits(of_ref.astype(np.float32))
+    o_f = to_dev_bf16(of_bits)
+    oc32 = oc_ref.astype(np.float32)
+    o_c = torch.from_numpy(oc32).cuda() if w.gated else None
     g_f = torch.from_numpy(x["g_f"]).cuda() if w.gated else None
     g_c = torch.from_numpy(x["g_c"]).cuda() if w.gated else None
-    out = torch.empty_like(q)
-    bufs = vsa.vsa_forward(shape, q, k, v, w.topk, out, g_f, g_c)
     rng = np.random.default_rng(w.seed + 100)
     dout_bits = wl.f32_to_bf16_bits(rng.standard_normal((B, H, N, d), dtype=np.float32))
     dout = to_dev_bf16(dout_bits)
-    dof = torch.full_like(bufs.o_f, 5.0)
+    dof = torch.full_like(o_f, 5.0)
     delta = torch.full((B, H, 64 * C), 5.0, dtype=torch.float32, device="cuda")
     doc = torch.empty(B, H, C, d, dtype=torch.float32, device="cuda") if w.gated else None
     dgf = torch.empty(B, H, N, dtype=torch.float32, device="cuda") if w.gated else None
     dgc = torch.empty_like(dgf) if w.gated else None
-    vsa.vsa_backward_prep(shape, dout, bufs.o_f, dof, delta, bufs.o_c if w.gated else None,
-                          g_f, g_c, doc, dgf, dgc)
+    vsa.vsa_backward_prep(shape, dout, o_f, dof, delta, o_c, g_f, g_c, doc, dgf, dgc)
     torch.cuda.synchronize()
     assert vsa.vsa_get_status() == 0
 
-    of = bf16_dev_to_f64(bufs.o_f)
-    oc = bufs.o_c.double().cpu().numpy() if w.gated else np.zeros((B, H, C, d))
+    of = vo.bf16_bits_to_f64(of_bits)
+    oc = oc32.astype(np.float64) if w.gated else np.zeros((B, H, C, d))
     dout64 = vo.bf16_bits_to_f64(dout_bits)
-    dout_t, counts = vo.tile_permute(dout64, w.grid)
+    dout_t, _ = vo.tile_permute(dout64, w.grid)
     gf64 = x["g_f"].astype(np.float64) if w.gated else None
     gc64 = x["g_c"].astype(np.float64) if w.gated else None
     dof_ref, doc_ref, dgf_ref, dgc_ref = vb.combine_backward(dout_t, of, oc, counts, w.grid, gf64, gc64)

@@ -1,14 +1,14 @@
 """vsa_select_transpose against the oracle's selection transpose, bit for bit
-(integer work): random ascending selections, the coarse stage's own selection
-on a ragged workload, every cube selected, and one key cube selected by all."""
+(integer work): random ascending selections, the oracle's coarse-stage
+selection on a ragged workload, every cube selected, and one key cube selected by all."""
 
 import numpy as np
 import pytest
 import torch
 
 from oracle import vsa_backward as vb
+from oracle import vsa_oracle as vo
 from video_dit_block_vsa_b200 import workloads as wl
-from tests.vsa_checks import to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -55,13 +55,14 @@ def test_one_key_cube_chosen_by_every_query(vsa):
 
 
 def test_coarse_stage_selection(vsa):
+    """A selection with the structure the coarse stage gives (the oracle's own
+    top-k on a ragged 480p grid): the lists' lengths spread unevenly."""
     w = wl.WORKLOADS["wan1.3b_480p_21x30x52"]
     x = wl.make_inputs(w, heads=2)
     shape = vsa.make_shape(w.batch, 2, w.head_dim, w.grid)
-    bufs = vsa.VsaBuffers(shape, w.topk)
-    for n, t in (("q", bufs.q_t), ("k", bufs.k_t), ("v", bufs.v_t)):
-        vsa.vsa_tile_permute(shape, to_dev_bf16(x[n]), t, bufs.counts if n == "q" else None)
-    vsa.vsa_coarse_select(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, w.topk, bufs.sel,
-                          bufs.workspace)
-    torch.cuda.synchronize()
-    run(vsa, shape, bufs.sel.cpu().numpy().astype(np.int64))
+    pooled = []
+    for n in ("q", "k", "v"):
+        t, counts = vo.tile_permute(vo.bf16_bits_to_f64(x[n]), w.grid)
+        pooled.append(vo.pool(t, counts))
+    S_c, _ = vo.coarse_attention(*pooled)
+    run(vsa, shape, vo.topk_select(S_c, w.topk))

@@ -119,6 +119,13 @@ def test_null_and_misaligned_pointers_rejected_before_launch(vsa):
     assert cp(ctypes.byref(s), 5, None, p, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
     assert cp(ctypes.byref(s), 2, None, None, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
     assert cp(ctypes.byref(s), 2, None, p, None, p, 16, None) == vsa.VSA_ERR_INVALID_ARG
+    cb = lib.vsa_coarse_backward
+    assert cb(ctypes.byref(s), None, p, p, p, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
+    assert cb(ctypes.byref(s), p, p, p, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
+    assert cb(ctypes.byref(s), p, p, odd, p, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
+    assert cb(ctypes.byref(s), p, p, p, p, ctypes.c_void_p(0x100010), 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
+    # 3 floats of statistics per (b, h, cube): 3 * 2 * 4 * 4 bytes here
+    assert cb(ctypes.byref(s), p, p, p, p, p, 3 * 2 * 4 * 4 - 1, None) == vsa.VSA_ERR_INVALID_ARG
     assert lib.vsa_debug_wait_timeout(10, None) == vsa.VSA_ERR_INVALID_ARG
 
 

@@ -32,6 +32,8 @@ cudaError_t launch_select_transpose(int, int, int, const int32_t*, int32_t*, int
                                     int*, cudaStream_t);
 cudaError_t launch_backward_prep(const Geom&, const void*, const void*, const float*, const float*,
                                  const float*, void*, float*, float*, float*, float*, cudaStream_t);
+cudaError_t launch_coarse_backward(int, int, int, const float*, const float*, const float*, float*,
+                                   float*, cudaStream_t);
 
 // Device-side status word, one per device that loads the library.
 __device__ int g_status;
@@ -400,6 +402,25 @@ int vsa_backward_prep(const vsa_shape* shape, const void* dout, const void* o_fi
                                       g_fine, g_coarse, do_fine_tiled, delta,
                                       gated ? do_coarse : nullptr, gated ? dg_fine : nullptr,
                                       gated ? dg_coarse : nullptr, stream));
+}
+
+int vsa_coarse_backward(const vsa_shape* shape, const float* pooled, const float* o_coarse,
+                        const float* do_coarse, float* d_pooled, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (!pooled || !o_coarse || !do_coarse || !d_pooled || !workspace) return VSA_ERR_INVALID_ARG;
+  if (!aligned16(pooled) || !aligned16(o_coarse) || !aligned16(do_coarse) || !aligned16(d_pooled) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return VSA_ERR_INVALID_ARG;
+  const long long bh = static_cast<long long>(g.B) * g.H;
+  if (bh > 65535) return VSA_ERR_UNSUPPORTED;  // (b, h) is the grid's y index
+  if (workspace_bytes < static_cast<size_t>(3 * bh * g.C) * sizeof(float)) return VSA_ERR_INVALID_ARG;
+  DeviceState* st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  return cuda_rc(launch_coarse_backward(static_cast<int>(bh), g.C, g.d, pooled, o_coarse, do_coarse,
+                                        d_pooled, static_cast<float*>(workspace), stream));
 }
 
 int vsa_get_status(cudaStream_t stream) {

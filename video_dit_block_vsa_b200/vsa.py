@@ -36,7 +36,7 @@ EXPORTED = ("vsa_num_cubes", "vsa_topk_from_ratio", "vsa_workspace_bytes", "vsa_
             "vsa_coarse_select_pooled", "vsa_coarse_select_noalloc",
             "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_out",
             "vsa_combine", "vsa_untile", "vsa_forward_host_workspace_bytes", "vsa_forward_host",
-            "vsa_select_transpose", "vsa_backward_prep", "vsa_get_status", "vsa_debug_wait_timeout",
+            "vsa_select_transpose", "vsa_backward_prep", "vsa_coarse_backward", "vsa_get_status", "vsa_debug_wait_timeout",
             "vsa_strerror")
 
 
@@ -76,6 +76,7 @@ _sig = {
                                         ctypes.c_int, _P]),
     "vsa_select_transpose": (ctypes.c_int, [_SP, _P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
     "vsa_backward_prep": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "vsa_coarse_backward": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "vsa_get_status": (ctypes.c_int, [_P]),
     "vsa_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
     "vsa_strerror": (ctypes.c_char_p, [ctypes.c_int]),
@@ -374,6 +375,27 @@ def vsa_backward_prep(shape, dout, o_fine_tiled, do_fine_tiled, delta, o_coarse=
                                   _ptr(g_fine), _ptr(g_coarse), _ptr(do_fine_tiled), _ptr(delta),
                                   _ptr(do_coarse), _ptr(dg_fine), _ptr(dg_coarse), _stream(stream)),
            "vsa_backward_prep")
+
+
+def vsa_coarse_backward(shape, pooled, o_coarse, do_coarse, d_pooled, workspace, stream=None):
+    """Gradients of the coarse attention w.r.t. the pooled vectors (see vsa.h)."""
+    B, H, N, d, C = _dims(shape)
+    _expect(pooled, torch.float32, (3, B, H, C, d), "pooled")
+    _expect(o_coarse, torch.float32, (B, H, C, d), "o_coarse")
+    _expect(do_coarse, torch.float32, (B, H, C, d), "do_coarse")
+    _expect(d_pooled, torch.float32, (3, B, H, C, d), "d_pooled")
+    _check(_lib.vsa_coarse_backward(ctypes.byref(shape), _ptr(pooled), _ptr(o_coarse), _ptr(do_coarse),
+                                    _ptr(d_pooled), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)),
+           "vsa_coarse_backward")
+
+
+def pooled_view(shape, workspace):
+    """The pooled qbar, kbar, vbar [3, B, H, C, d] float32 at the start of a
+    vsa_tile_permute_pool / vsa_coarse_select workspace (a view, no copy)."""
+    B, H, N, d, C = _dims(shape)
+    n = 3 * B * H * C * d
+    return workspace.view(torch.uint8)[: 4 * n].view(torch.float32).view(3, B, H, C, d)
 
 
 def vsa_get_status(stream=None) -> int:
