@@ -421,6 +421,88 @@ TMA_INGEST_GBS_PER_SM = 99.3
 # (b, h) planes per chunk of the host-buffer path in the end-to-end leg.
 HOST_CHUNK_HEADS = 2
 
+def run_backward_pieces(args, w):
+    """Times the backward pieces built so far on the workload (one GPU, not the
+    default bench line): the combine-gradient prep pass, the selection
+    transpose and the coarse attention backward, each after a forward that
+    leaves O_f tiled, the selection and O_c resident.  Prints one JSON line."""
+    import torch
+
+    from video_dit_block_vsa_b200 import vsa
+
+    x = wl.make_inputs(w)
+    shape = vsa.make_shape(w.batch, w.heads, w.head_dim, w.grid)
+    dev = torch.device("cuda", 0)
+    to_dev = lambda b: torch.from_numpy(b.view(np.int16)).to(dev).view(torch.bfloat16)
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    B, H, N, d, C = w.batch, w.heads, w.tokens, w.head_dim, w.cubes
+    bufs = vsa.VsaBuffers(shape, w.topk, device=dev, want_lse=True)
+    vsa.vsa_tile_permute_pool(shape, q, k, v, bufs.q_t, bufs.k_t, bufs.v_t, bufs.workspace,
+                              bufs.counts)
+    vsa.vsa_coarse_select_pooled(shape, w.topk, bufs.sel, bufs.workspace, o_coarse=bufs.o_c)
+    vsa.vsa_block_sparse_fwd(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, bufs.sel, w.topk,
+                             bufs.o_f, bufs.lse)
+    rng = np.random.default_rng(w.seed + 1)
+    dout = to_dev(wl.f32_to_bf16_bits(rng.standard_normal((B, H, N, d), dtype=np.float32)))
+    g_f = torch.full((B, H, N), 0.5, dtype=torch.float32, device=dev)
+    g_c = torch.full((B, H, N), 0.5, dtype=torch.float32, device=dev)
+    dof = torch.empty_like(bufs.o_f)
+    delta = torch.empty(B, H, 64 * C, dtype=torch.float32, device=dev)
+    doc = torch.empty(B, H, C, d, dtype=torch.float32, device=dev)
+    dgf = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    dgc = torch.empty_like(dgf)
+    offs = torch.empty(B, H, C + 1, dtype=torch.int32, device=dev)
+    lists = torch.empty(B, H, C * w.topk, dtype=torch.int32, device=dev)
+    t_ws = torch.empty(B * H * C * w.topk * 4, dtype=torch.uint8, device=dev)
+    d_pooled = torch.empty(3, B, H, C, d, dtype=torch.float32, device=dev)
+    c_ws = torch.empty(3 * B * H * C * 4, dtype=torch.uint8, device=dev)
+    pooled = vsa.pooled_view(shape, bufs.workspace)
+    stream = torch.cuda.current_stream()
+    pieces = {
+        "backward_prep": lambda: vsa.vsa_backward_prep(shape, dout, bufs.o_f, dof, delta, bufs.o_c,
+                                                       g_f, g_c, doc, dgf, dgc),
+        "select_transpose": lambda: vsa.vsa_select_transpose(shape, bufs.sel, w.topk, offs, lists,
+                                                             t_ws),
+        "coarse_backward": lambda: vsa.vsa_coarse_backward(shape, pooled, bufs.o_c, doc, d_pooled,
+                                                           c_ws),
+    }
+    ms = {}
+    for name, fn in pieces.items():
+        for _ in range(max(args.warmup, 1)):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms[name] = a.elapsed_time(b) / args.steps
+    status = vsa.vsa_get_status()
+    if status != 0:
+        raise RuntimeError(f"device status: {vsa.vsa_strerror(status)}")
+    peaks = load_peaks()
+    valid = N * B * H  # valid rows over all (b, h)
+    # prep: dout, O_f (valid rows), gates read; dO_f, delta (all 64*C rows),
+    # dO_c, dg_f, dg_c written
+    prep_bytes = (valid * d * 2 * 2 + valid * 4 * 2 + B * H * 64 * C * (d * 2 + 4)
+                  + B * H * C * d * 4 + valid * 4 * 2 + B * H * C * d * 4)
+    # coarse backward: the 5 C x C x d products (S, dP, dQ, dK, dV) of a
+    # backward, 2 flops each multiply-add
+    coarse_flops = 10.0 * B * H * C * C * d
+    line = {"mode": "backward_pieces", "workload": w.name, "steps": args.steps,
+            "warmup": args.warmup, "ms": {k_: round(v_, 4) for k_, v_ in ms.items()},
+            "backward_prep": {"algorithmic_bytes": prep_bytes,
+                              "achieved_gbs": round(prep_bytes / ms["backward_prep"] / 1e6, 1),
+                              "peak_gbs": peaks["hbm"], "peak_source": peaks["source"],
+                              "gated": True},
+            "coarse_backward": {"algorithmic_flops": coarse_flops,
+                                "achieved_tflops": round(coarse_flops / ms["coarse_backward"] / 1e9, 2),
+                                "dtype": "f32", "note": "SIMT float32, two passes"}}
+    print(json.dumps(line))
+    return 0
+
+
 # Revision tag of the fine kernel; ncu traffic figures are only reported for
 # the revision they were captured on.
 KERNEL_REV = "fine-v3.2-out"
@@ -435,8 +517,12 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward-pieces", action="store_true",
+                    help="time the backward pieces built so far instead (one GPU)")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.workload]
+    if args.backward_pieces:
+        return run_backward_pieces(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)
