@@ -455,7 +455,7 @@ def run_backward_pieces(args, w):
     lists = torch.empty(B, H, C * w.topk, dtype=torch.int32, device=dev)
     t_ws = torch.empty(B * H * C * w.topk * 4, dtype=torch.uint8, device=dev)
     d_pooled = torch.empty(3, B, H, C, d, dtype=torch.float32, device=dev)
-    c_ws = torch.empty(3 * B * H * C * 4, dtype=torch.uint8, device=dev)
+    c_ws = torch.empty(vsa.vsa_coarse_backward_workspace_bytes(shape), dtype=torch.uint8, device=dev)
     pooled = vsa.pooled_view(shape, bufs.workspace)
     stream = torch.cuda.current_stream()
     pieces = {
@@ -498,7 +498,7 @@ def run_backward_pieces(args, w):
                               "gated": True},
             "coarse_backward": {"algorithmic_flops": coarse_flops,
                                 "achieved_tflops": round(coarse_flops / ms["coarse_backward"] / 1e9, 2),
-                                "dtype": "f32", "note": "SIMT float32, two passes"}}
+                                "dtype": "f32", "note": "SIMT float32 register-tiled products"}}
     print(json.dumps(line))
     return 0
 

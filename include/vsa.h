@@ -286,6 +286,11 @@ int vsa_backward_prep(const vsa_shape* shape, const void* dout, const void* o_fi
                       void* do_fine_tiled, float* delta, float* do_coarse, float* dg_fine,
                       float* dg_coarse, cudaStream_t stream);
 
+/* Bytes of workspace vsa_coarse_backward needs to process all B*H planes in
+ * one pass: B*H * 2*C*ldc*4, ldc = C rounded up to a multiple of 64 (two C x C
+ * float32 matrices per plane).  0 for an invalid shape. */
+size_t vsa_coarse_backward_workspace_bytes(const vsa_shape* shape);
+
 /* Backward of the coarse attention O_c = softmax(qbar kbar^T / sqrt(d)) vbar
  * (the coarse stage of vsa_coarse_select; the pages describe no backward, this
  * differentiates that forward exactly, in float32):
@@ -295,11 +300,11 @@ int vsa_backward_prep(const vsa_shape* shape, const void* dout, const void* o_fi
  *   o_coarse  float32 [B, H, C, d]: the forward's O_c (read)
  *   do_coarse float32 [B, H, C, d]: gradient of O_c, e.g. from vsa_backward_prep (read)
  *   d_pooled  float32 [3, B, H, C, d]: dqbar, dkbar, dvbar (written)
- *   workspace device scratch of at least 3*B*H*C*4 bytes, 256-byte aligned
- *             (per query cube: the row max, 1/z and <do_coarse, o_coarse>)
- * All float pointers 16-byte aligned; B*H at most 65535.  No C x C matrix is
- * stored: a row pass gives dqbar and the softmax statistics, a column pass
- * recomputes P from them for dkbar and dvbar. */
+ *   workspace device scratch, 256-byte aligned, holding P and dS of as many
+ *             planes as fit: at least one plane's share of
+ *             vsa_coarse_backward_workspace_bytes (2*C*ldc*4 bytes); with less
+ *             than the full size the planes are processed in chunks
+ * All float pointers 16-byte aligned; B*H at most 65535. */
 int vsa_coarse_backward(const vsa_shape* shape, const float* pooled, const float* o_coarse,
                         const float* do_coarse, float* d_pooled, void* workspace,
                         size_t workspace_bytes, cudaStream_t stream);

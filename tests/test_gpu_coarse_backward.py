@@ -51,16 +51,18 @@ def check(got, refs, what):
         assert e.mean() <= MEAN_REL * m, f"{what} {name}: mean err {e.mean():.3e}"
 
 
-CASES = [
-    (wl.WORKLOADS["tiny_k2"], 2),                                             # C = 4, d = 64
-    (wl.Workload("ragged_d64", 2, 2, 64, (16, 36, 36), 8, 31, 0.5, False), None),  # C = 324
-    (wl.WORKLOADS["wan1.3b_ft_16x28x52"], 2),                                 # C = 364, d = 128
-    (wl.WORKLOADS["wan14b_720p_21x45x80_k180"], 1),                           # C = 1440
+CASES = [  # (workload, heads, one plane of workspace)
+    (wl.WORKLOADS["tiny_k2"], 2, None),                                        # C = 4, d = 64
+    (wl.Workload("ragged_d64", 2, 2, 64, (16, 36, 36), 8, 31, 0.5, False), None, True),  # C = 324
+    (wl.Workload("odd_c27", 1, 3, 128, (9, 10, 11), 5, 32, 0.5, False), None, None),  # C = 27
+    (wl.WORKLOADS["wan1.3b_ft_16x28x52"], 2, None),                            # C = 364, d = 128
+    (wl.WORKLOADS["wan14b_720p_21x45x80_k180"], 2, True),                      # C = 1440
 ]
 
 
-@pytest.mark.parametrize("w,heads", CASES, ids=[c[0].name for c in CASES])
-def test_coarse_backward_matches_oracle(vsa, w, heads):
+@pytest.mark.parametrize("w,heads,chunked", CASES,
+                         ids=[c[0].name + ("-chunked" if c[2] else "") for c in CASES])
+def test_coarse_backward_matches_oracle(vsa, w, heads, chunked):
     H = w.heads if heads is None else heads
     B, d = w.batch, w.head_dim
     _, pooled = oracle_pooled(w, H)
@@ -76,7 +78,9 @@ def test_coarse_backward_matches_oracle(vsa, w, heads):
     shape = vsa.make_shape(B, H, d, w.grid)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     d_pooled = torch.full((3, B, H, C, d), float("nan"), dtype=torch.float32, device="cuda")
-    ws = torch.empty(3 * B * H * C * 4, dtype=torch.uint8, device="cuda")
+    full = vsa.vsa_coarse_backward_workspace_bytes(shape)
+    # the whole workspace, or one plane's share (the planes then run in chunks)
+    ws = torch.empty(full if chunked is None else full // (B * H), dtype=torch.uint8, device="cuda")
     vsa.vsa_coarse_backward(shape, dev(np.stack(p32)), dev(oc32), dev(doc32), d_pooled, ws)
     torch.cuda.synchronize()
     assert vsa.vsa_get_status() == 0
@@ -99,9 +103,9 @@ def test_coarse_backward_on_the_forward_workspace(vsa):
                               bufs.counts)
     vsa.vsa_coarse_select_pooled(shape, w.topk, bufs.sel, bufs.workspace, o_coarse=bufs.o_c)
     d_pooled = torch.full((3, B, H, C, d), float("nan"), dtype=torch.float32, device="cuda")
-    stats = torch.empty(3 * B * H * C * 4, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(vsa.vsa_coarse_backward_workspace_bytes(shape), dtype=torch.uint8, device="cuda")
     vsa.vsa_coarse_backward(shape, vsa.pooled_view(shape, bufs.workspace), bufs.o_c,
-                            torch.from_numpy(doc32).cuda(), d_pooled, stats)
+                            torch.from_numpy(doc32).cuda(), d_pooled, ws)
     torch.cuda.synchronize()
     assert vsa.vsa_get_status() == 0
     check(d_pooled.cpu().numpy(), refs, "forward workspace")

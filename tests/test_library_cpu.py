@@ -124,8 +124,11 @@ def test_null_and_misaligned_pointers_rejected_before_launch(vsa):
     assert cb(ctypes.byref(s), p, p, p, None, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
     assert cb(ctypes.byref(s), p, p, odd, p, p, 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
     assert cb(ctypes.byref(s), p, p, p, p, ctypes.c_void_p(0x100010), 1 << 20, None) == vsa.VSA_ERR_INVALID_ARG
-    # 3 floats of statistics per (b, h, cube): 3 * 2 * 4 * 4 bytes here
-    assert cb(ctypes.byref(s), p, p, p, p, p, 3 * 2 * 4 * 4 - 1, None) == vsa.VSA_ERR_INVALID_ARG
+    # less than one plane's P and dS (C = 4, row stride 64): 2 * 4 * 64 * 4 bytes
+    assert cb(ctypes.byref(s), p, p, p, p, p, 2 * 4 * 64 * 4 - 1, None) == vsa.VSA_ERR_INVALID_ARG
+    assert vsa.vsa_coarse_backward_workspace_bytes(s) == 2 * (2 * 4 * 64 * 4)
+    big = vsa.make_shape(1, 40, 128, (21, 45, 80))  # C = 1440, row stride 1472
+    assert vsa.vsa_coarse_backward_workspace_bytes(big) == 40 * 2 * 1440 * 1472 * 4
     assert lib.vsa_debug_wait_timeout(10, None) == vsa.VSA_ERR_INVALID_ARG
 
 

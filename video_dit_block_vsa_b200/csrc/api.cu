@@ -33,7 +33,8 @@ cudaError_t launch_select_transpose(int, int, int, const int32_t*, int32_t*, int
 cudaError_t launch_backward_prep(const Geom&, const void*, const void*, const float*, const float*,
                                  const float*, void*, float*, float*, float*, float*, cudaStream_t);
 cudaError_t launch_coarse_backward(int, int, int, const float*, const float*, const float*, float*,
-                                   float*, cudaStream_t);
+                                   void*, size_t, cudaStream_t);
+size_t coarse_backward_plane_bytes(int C);
 
 // Device-side status word, one per device that loads the library.
 __device__ int g_status;
@@ -404,6 +405,12 @@ int vsa_backward_prep(const vsa_shape* shape, const void* dout, const void* o_fi
                                       gated ? dg_coarse : nullptr, stream));
 }
 
+size_t vsa_coarse_backward_workspace_bytes(const vsa_shape* shape) {
+  Geom g;
+  if (make_geom(shape, &g) != VSA_OK) return 0;
+  return static_cast<size_t>(g.B) * g.H * coarse_backward_plane_bytes(g.C);
+}
+
 int vsa_coarse_backward(const vsa_shape* shape, const float* pooled, const float* o_coarse,
                         const float* do_coarse, float* d_pooled, void* workspace,
                         size_t workspace_bytes, cudaStream_t stream) {
@@ -415,12 +422,12 @@ int vsa_coarse_backward(const vsa_shape* shape, const float* pooled, const float
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return VSA_ERR_INVALID_ARG;
   const long long bh = static_cast<long long>(g.B) * g.H;
-  if (bh > 65535) return VSA_ERR_UNSUPPORTED;  // (b, h) is the grid's y index
-  if (workspace_bytes < static_cast<size_t>(3 * bh * g.C) * sizeof(float)) return VSA_ERR_INVALID_ARG;
+  if (bh > 65535) return VSA_ERR_UNSUPPORTED;  // (b, h) is a grid index
+  if (workspace_bytes < coarse_backward_plane_bytes(g.C)) return VSA_ERR_INVALID_ARG;
   DeviceState* st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_coarse_backward(static_cast<int>(bh), g.C, g.d, pooled, o_coarse, do_coarse,
-                                        d_pooled, static_cast<float*>(workspace), stream));
+                                        d_pooled, workspace, workspace_bytes, stream));
 }
 
 int vsa_get_status(cudaStream_t stream) {

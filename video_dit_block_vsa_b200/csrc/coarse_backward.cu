@@ -3,20 +3,18 @@
 // backward pass.  With P the softmax, dO_c the incoming gradient and
 // scale = 1/sqrt(d):
 //   D_i   = <dO_c[i], O_c[i]>
-//   dS_ij = P_ij (<dO_c[i], vbar[j]> - D_i)
-//   dqbar[i] = scale sum_j dS_ij kbar[j]
-//   dkbar[j] = scale sum_i dS_ij qbar[i],   dvbar[j] = sum_i P_ij dO_c[i]
+//   dS_ij = P_ij (dP_ij - D_i),   dP = dO_c vbar^T
+//   dqbar = scale dS kbar,   dkbar = scale dS^T qbar,   dvbar = P^T dO_c
 //
-// Two passes, no C x C matrix in memory:
-//   rows    (one CTA per query cube i): the row of logits in shared memory,
-//           its max m_i and 1/z_i, D_i, the row of dS, then dqbar[i];
-//           m, 1/z and D go to a 3*B*H*C float scratch.
-//   columns (one CTA per key cube j): recomputes column j of P from the saved
-//           m and 1/z with the same float arithmetic (so P is bit-identical
-//           to the rows pass), forms column j of dS, then dkbar[j], dvbar[j].
-// Each thread takes whole dot products of length d (float4 loads of one row);
-// the weighted sums over rows run with consecutive threads on consecutive
-// elements of a row, so those loads are coalesced.
+// C is at most 8192 (1440 for a 720p video), so the C x C matrices are kept in
+// a workspace (row stride ldc = C rounded up to 64, pad columns zero):
+//   logits  (64 x 64 tiles)  S = scale qbar kbar^T into buffer 0, dP into buffer 1
+//   softmax (a warp per row) P over buffer 0, dS over buffer 1, D from O_c
+//   grads   (64 x d tiles)   dqbar, dkbar, dvbar: products over the C rows
+// The two tile kernels are register-tiled SIMT GEMMs: 256 threads, 32-deep
+// k chunks staged k-major in shared memory, each thread 4 rows x (BN/16)
+// columns.  Float32 throughout: the sums are those of the definition, in
+// float32 order.  The (b, h) planes run in chunks as large as the workspace.
 #include <cmath>
 
 #include "common.cuh"
@@ -26,177 +24,254 @@ namespace vsa {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kTileM = 64;  // rows of an output tile
+constexpr int kChunk = 32;  // k per staged chunk
 
-__device__ __forceinline__ float block_reduce(float v, float* red, bool is_max) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// One operand chunk into shared memory, k-major: dst[k][m] for k < 32, m < W.
+// kKContig: element (m, k) at src[m * ld + k]  (rows of the operand are m;
+//           valid while m < mlim; k stays inside the row by construction)
+// else:     element (m, k) at src[k * ld + m]  (valid while k < klim)
+// Invalid elements load as 0.  Every float4 read is 16-byte aligned: ld, the
+// chunk start and the tile start are multiples of 4 floats.
+template <int W, bool kKContig>
+__device__ __forceinline__ void stage(float* dst, const float* __restrict__ src, int ld, int m0,
+                                      int mlim, int k0, int klim) {
+  if constexpr (kKContig) {
+    // W rows x 8 float4 of k; consecutive threads take consecutive rows so
+    // the transposed shared-memory stores hit consecutive banks
+    for (int idx = threadIdx.x; idx < W * (kChunk / 4); idx += kThreads) {
+      const int m = idx % W, kq = idx / W;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (m0 + m < mlim)
+        x = __ldg(reinterpret_cast<const float4*>(src + static_cast<long long>(m0 + m) * ld + k0 + 4 * kq));
+      dst[(4 * kq + 0) * W + m] = x.x;
+      dst[(4 * kq + 1) * W + m] = x.y;
+      dst[(4 * kq + 2) * W + m] = x.z;
+      dst[(4 * kq + 3) * W + m] = x.w;
+    }
+  } else {
+    // 32 rows of k x W/4 float4 of m: coalesced reads, float4 stores
+    for (int idx = threadIdx.x; idx < kChunk * (W / 4); idx += kThreads) {
+      const int m4 = idx % (W / 4), k = idx / (W / 4);
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (k0 + k < klim)
+        x = __ldg(reinterpret_cast<const float4*>(src + static_cast<long long>(k0 + k) * ld + m0 + 4 * m4));
+      *reinterpret_cast<float4*>(&dst[k * W + 4 * m4]) = x;
+    }
+  }
+}
+
+// Column of the c-th accumulator of thread tx in a BN-wide tile: two float4
+// groups 64 apart when BN = 128, so a quarter warp reads 128 contiguous bytes.
+__device__ __forceinline__ int tile_col(int tx, int c) { return (c >> 2) * 64 + tx * 4 + (c & 3); }
+
+// acc[r][c] += sum over the chunk of As[k][ty*4 + r] * Bs[k][tile_col(tx, c)].
+template <int BN>
+__device__ __forceinline__ void chunk_fma(const float* As, const float* Bs, int tx, int ty,
+                                          float (&acc)[4][BN / 16]) {
+#pragma unroll 8
+  for (int k = 0; k < kChunk; ++k) {
+    const float4 a = *reinterpret_cast<const float4*>(&As[k * kTileM + ty * 4]);
+    const float av[4] = {a.x, a.y, a.z, a.w};
+    float bv[BN / 16];
+#pragma unroll
+    for (int g = 0; g < BN / 64; ++g) {
+      const float4 b = *reinterpret_cast<const float4*>(&Bs[k * BN + g * 64 + tx * 4]);
+      bv[4 * g] = b.x; bv[4 * g + 1] = b.y; bv[4 * g + 2] = b.z; bv[4 * g + 3] = b.w;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < BN / 16; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+  }
+}
+
+// out[i][j] = mul * sum_e A[i][e] B[j][e] for a 64 x 64 tile (A, B rows of d floats).
+template <int D>
+__device__ __forceinline__ void logits_tile(const float* __restrict__ A, const float* __restrict__ B,
+                                            int C, int ldc, int i0, int j0, float mul,
+                                            float* __restrict__ out, float* As, float* Bs) {
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int e0 = 0; e0 < D; e0 += kChunk) {
+    __syncthreads();  // the previous chunk (or tile) is no longer read
+    stage<kTileM, true>(As, A, D, i0, C, e0, D);
+    stage<kTileM, true>(Bs, B, D, j0, C, e0, D);
+    __syncthreads();
+    chunk_fma<64>(As, Bs, tx, ty, acc);
+  }
+  // rows i < C; columns j0..j0+63 lie inside the padded row (j >= C are 0:
+  // their operand rows were staged as zeros)
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int i = i0 + ty * 4 + r;
+    if (i >= C) continue;
+    float* row = out + static_cast<long long>(i) * ldc + j0 + tx * 4;
+    *reinterpret_cast<float4*>(row) =
+        make_float4(acc[r][0] * mul, acc[r][1] * mul, acc[r][2] * mul, acc[r][3] * mul);
+  }
+}
+
+// grid (ldc/64 key tiles, ldc/64 query tiles, planes of this chunk).
+template <int D>
+__global__ void __launch_bounds__(kThreads) coarse_bwd_logits(
+    int C, int ldc, const float* __restrict__ qb, const float* __restrict__ kb,
+    const float* __restrict__ vb, const float* __restrict__ doc, float* __restrict__ sbuf,
+    float* __restrict__ dpbuf) {
+  __shared__ __align__(16) float As[kChunk * kTileM];
+  __shared__ __align__(16) float Bs[kChunk * kTileM];
+  const long long bh = blockIdx.z;
+  const long long plane = bh * C * D;
+  const long long mat = bh * C * static_cast<long long>(ldc);
+  const int i0 = blockIdx.y * kTileM, j0 = blockIdx.x * kTileM;
+  const float scale = 1.0f / sqrtf(static_cast<float>(D));
+  logits_tile<D>(qb + plane, kb + plane, C, ldc, i0, j0, scale, sbuf + mat, As, Bs);
+  logits_tile<D>(doc + plane, vb + plane, C, ldc, i0, j0, 1.0f, dpbuf + mat, As, Bs);
+}
+
+// grid (ceil(C/8), planes): one warp per row i.  Turns the row of S into P and
+// the row of dP into dS in place; pad columns stay 0.
+__global__ void __launch_bounds__(kThreads) coarse_bwd_softmax(
+    int C, int ldc, int d, const float* __restrict__ oc, const float* __restrict__ doc,
+    float* __restrict__ sbuf, float* __restrict__ dpbuf) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i = blockIdx.x * (kThreads / 32) + warp;
+  if (i >= C) return;  // whole warp
+  const long long bh = blockIdx.y;
+  const long long r = (bh * C + i) * static_cast<long long>(ldc);
+  float* s = sbuf + r;
+  float* dp = dpbuf + r;
+  // online max and sum per lane, then merged across the warp
+  float m = -INFINITY, z = 0.f;
+  for (int j = lane; j < C; j += 32) {
+    const float x = s[j];
+    if (x > m) {
+      z = z * expf(m - x) + 1.0f;  // m = -inf on the first element: z = 0 * 0 + 1
+      m = x;
+    } else {
+      z += expf(x - m);
+    }
+  }
   for (int off = 16; off; off >>= 1) {
-    const float o = __shfl_xor_sync(0xffffffffu, v, off);
-    v = is_max ? fmaxf(v, o) : v + o;
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+    const float z2 = __shfl_xor_sync(0xffffffffu, z, off);
+    const float mn = fmaxf(m, m2);
+    // a lane that saw no element has m = -inf, z = 0 and contributes nothing
+    const float a = (m == -INFINITY) ? 0.f : z * expf(m - mn);
+    const float b = (m2 == -INFINITY) ? 0.f : z2 * expf(m2 - mn);
+    z = a + b;
+    m = mn;
   }
-  __syncthreads();  // red[] may still be read from the previous reduction
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  float r = red[0];
-  for (int w = 1; w < kThreads / 32; ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
-  return r;
-}
-
-// <a, row> over d elements: a in shared memory, row in global memory (16-byte aligned).
-__device__ __forceinline__ float dot_row(const float* a, const float* __restrict__ row, int d) {
-  const float4* r4 = reinterpret_cast<const float4*>(row);
-  float s = 0.f;
-  for (int e = 0; e < (d >> 2); ++e) {
-    const float4 x = __ldg(&r4[e]);
-    s = fmaf(a[4 * e], x.x, s);
-    s = fmaf(a[4 * e + 1], x.y, s);
-    s = fmaf(a[4 * e + 2], x.z, s);
-    s = fmaf(a[4 * e + 3], x.w, s);
-  }
-  return s;
-}
-
-// out[e] = mul * sum_{r < n} w[r] M[r, e] for e < d (w in shared memory, M global
-// [n][d]).  kThreads/d row groups sum interleaved rows; part[] combines them.
-// Must be called by the whole block; out is written by threads e < d.
-__device__ __forceinline__ void weighted_rows(const float* w, const float* __restrict__ M, int n,
-                                              int d, float mul, float* part,
-                                              float* __restrict__ out) {
-  const int groups = kThreads / d;
-  const int e = threadIdx.x % d, grp = threadIdx.x / d;
-  float acc = 0.f;
-  if (grp < groups)
-    for (int r = grp; r < n; r += groups) acc = fmaf(w[r], __ldg(&M[static_cast<long long>(r) * d + e]), acc);
-  __syncthreads();  // part[] may still be read from the previous call
-  part[threadIdx.x] = acc;
-  __syncthreads();
-  if (threadIdx.x < d) {
-    float s = 0.f;
-    for (int g = 0; g < groups; ++g) s += part[g * d + threadIdx.x];
-    out[threadIdx.x] = s * mul;
-  }
-}
-
-// grid (C, B*H).  Dynamic smem: qbar[i], dO_c[i] (d floats each), w[C].
-__global__ void __launch_bounds__(kThreads) coarse_bwd_rows(
-    int C, int d, const float* __restrict__ qb, const float* __restrict__ kb,
-    const float* __restrict__ vb, const float* __restrict__ oc, const float* __restrict__ doc,
-    float* __restrict__ dqb, float* __restrict__ row_max, float* __restrict__ row_rz,
-    float* __restrict__ row_D) {
-  extern __shared__ float sm[];
-  float* qi = sm;
-  float* gi = sm + d;
-  float* w = sm + 2 * d;
-  __shared__ float red[kThreads / 32];
-  __shared__ float part[kThreads];
-  const int i = blockIdx.x;
-  const long long bh = blockIdx.y;
-  const long long base = bh * C * static_cast<long long>(d);
-  const long long row_i = base + static_cast<long long>(i) * d;
-  const float scale = 1.0f / sqrtf(static_cast<float>(d));
-  float dpart = 0.f;
-  for (int e = threadIdx.x; e < d; e += kThreads) {
-    qi[e] = qb[row_i + e];
-    gi[e] = doc[row_i + e];
-    dpart = fmaf(gi[e], oc[row_i + e], dpart);
-  }
-  const float D = block_reduce(dpart, red, false);  // its barriers publish qi, gi
-  float mx = -INFINITY;
-  for (int j = threadIdx.x; j < C; j += kThreads) {
-    const float s = dot_row(qi, kb + base + static_cast<long long>(j) * d, d) * scale;
-    w[j] = s;
-    mx = fmaxf(mx, s);
-  }
-  mx = block_reduce(mx, red, true);
-  float z = 0.f;
-  for (int j = threadIdx.x; j < C; j += kThreads) {
-    const float p = expf(w[j] - mx);
-    w[j] = p;
-    z += p;
-  }
-  z = block_reduce(z, red, false);
+  const long long orow = (bh * C + i) * static_cast<long long>(d);
+  float D = 0.f;
+  for (int e = lane; e < d; e += 32) D = fmaf(doc[orow + e], oc[orow + e], D);
+  for (int off = 16; off; off >>= 1) D += __shfl_xor_sync(0xffffffffu, D, off);
   const float rz = 1.0f / z;
-  for (int j = threadIdx.x; j < C; j += kThreads) {
-    const float p = w[j] * rz;
-    const float dp = dot_row(gi, vb + base + static_cast<long long>(j) * d, d);
-    w[j] = p * (dp - D);  // dS_ij
-  }
-  __syncthreads();
-  weighted_rows(w, kb + base, C, d, scale, part, dqb + row_i);
-  if (threadIdx.x == 0) {
-    const long long r = bh * C + i;
-    row_max[r] = mx;
-    row_rz[r] = rz;
-    row_D[r] = D;
+  for (int j = lane; j < C; j += 32) {
+    const float p = expf(s[j] - m) * rz;
+    const float g = p * (dp[j] - D);
+    s[j] = p;
+    dp[j] = g;
   }
 }
 
-// grid (C, B*H).  Dynamic smem: kbar[j], vbar[j] (d floats each), p[C], ds[C].
-__global__ void __launch_bounds__(kThreads) coarse_bwd_cols(
-    int C, int d, const float* __restrict__ qb, const float* __restrict__ kb,
-    const float* __restrict__ vb, const float* __restrict__ doc, const float* __restrict__ row_max,
-    const float* __restrict__ row_rz, const float* __restrict__ row_D, float* __restrict__ dkb,
-    float* __restrict__ dvb) {
-  extern __shared__ float sm[];
-  float* kj = sm;
-  float* vj = sm + d;
-  float* p = sm + 2 * d;
-  float* ds = p + C;
-  __shared__ float part[kThreads];
-  const int j = blockIdx.x;
+// grid (ldc/64 row tiles, planes, 3): which = 0 dqbar = scale dS kbar,
+// 1 dkbar = scale dS^T qbar, 2 dvbar = P^T dO_c; each a 64 x D tile summed over
+// the C rows of the products' inner index.
+template <int D>
+__global__ void __launch_bounds__(kThreads) coarse_bwd_grads(
+    int C, int ldc, const float* __restrict__ qb, const float* __restrict__ kb,
+    const float* __restrict__ doc, const float* __restrict__ pbuf,
+    const float* __restrict__ dsbuf, float* __restrict__ dq, float* __restrict__ dk,
+    float* __restrict__ dv) {
+  __shared__ __align__(16) float As[kChunk * kTileM];
+  __shared__ __align__(16) float Bs[kChunk * D];
+  const int which = blockIdx.z;
   const long long bh = blockIdx.y;
-  const long long base = bh * C * static_cast<long long>(d);
-  const long long row_j = base + static_cast<long long>(j) * d;
-  const float scale = 1.0f / sqrtf(static_cast<float>(d));
-  for (int e = threadIdx.x; e < d; e += kThreads) {
-    kj[e] = kb[row_j + e];
-    vj[e] = vb[row_j + e];
+  const long long plane = bh * C * D;
+  const long long mat = bh * C * static_cast<long long>(ldc);
+  const int m0 = blockIdx.x * kTileM;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const float scale = 1.0f / sqrtf(static_cast<float>(D));
+  const float* A = (which == 2 ? pbuf : dsbuf) + mat;
+  const float* B = (which == 0 ? kb : which == 1 ? qb : doc) + plane;
+  float* out = (which == 0 ? dq : which == 1 ? dk : dv) + plane;
+  const float mul = which == 2 ? 1.0f : scale;
+  float acc[4][D / 16] = {};
+  for (int k0 = 0; k0 < C; k0 += kChunk) {
+    __syncthreads();
+    if (which == 0)  // A[i][j] = dS[i][j]: rows i, k = j contiguous (pads are 0)
+      stage<kTileM, true>(As, A, ldc, m0, C, k0, C);
+    else  // A[j][i] = dS[i][j] or P[i][j]: k = i indexes the rows
+      stage<kTileM, false>(As, A, ldc, m0, C, k0, C);
+    stage<D, false>(Bs, B, D, 0, D, k0, C);
+    __syncthreads();
+    chunk_fma<D>(As, Bs, tx, ty, acc);
   }
-  __syncthreads();
-  for (int i = threadIdx.x; i < C; i += kThreads) {
-    const long long r = bh * C + i;
-    // same operands and order as the rows pass: fmaf(a, b, c) == fmaf(b, a, c)
-    const float s = dot_row(kj, qb + base + static_cast<long long>(i) * d, d) * scale;
-    const float pij = expf(s - row_max[r]) * row_rz[r];
-    const float dp = dot_row(vj, doc + base + static_cast<long long>(i) * d, d);
-    p[i] = pij;
-    ds[i] = pij * (dp - row_D[r]);
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int m = m0 + ty * 4 + r;
+    if (m >= C) continue;
+    float* row = out + static_cast<long long>(m) * D;
+#pragma unroll
+    for (int g = 0; g < D / 64; ++g)
+      *reinterpret_cast<float4*>(row + tile_col(tx, 4 * g)) =
+          make_float4(acc[r][4 * g] * mul, acc[r][4 * g + 1] * mul, acc[r][4 * g + 2] * mul,
+                      acc[r][4 * g + 3] * mul);
   }
-  __syncthreads();
-  weighted_rows(ds, qb + base, C, d, scale, part, dkb + row_j);
-  weighted_rows(p, doc + base, C, d, 1.0f, part, dvb + row_j);
+}
+
+template <int D>
+cudaError_t run_chunk(int nbh, int C, int ldc, const float* qb, const float* kb, const float* vb,
+                      const float* oc, const float* doc, float* dq, float* dk, float* dv,
+                      float* sbuf, float* dpbuf, cudaStream_t s) {
+  const int tiles = ldc / kTileM;
+  coarse_bwd_logits<D><<<dim3(tiles, tiles, nbh), kThreads, 0, s>>>(C, ldc, qb, kb, vb, doc, sbuf,
+                                                                   dpbuf);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  coarse_bwd_softmax<<<dim3((C + 7) / 8, nbh), kThreads, 0, s>>>(C, ldc, D, oc, doc, sbuf, dpbuf);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  coarse_bwd_grads<D><<<dim3(tiles, nbh, 3), kThreads, 0, s>>>(C, ldc, qb, kb, doc, sbuf, dpbuf,
+                                                               dq, dk, dv);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t coarse_backward_smem_bytes(int C, int d) {
-  return static_cast<size_t>(2 * d + 2 * C) * sizeof(float);
+// Row stride of the workspace matrices and the bytes one (b, h) plane needs.
+int coarse_backward_ldc(int C) { return (C + kTileM - 1) / kTileM * kTileM; }
+
+size_t coarse_backward_plane_bytes(int C) {
+  return 2ull * static_cast<size_t>(C) * coarse_backward_ldc(C) * sizeof(float);
 }
 
 cudaError_t launch_coarse_backward(int BH, int C, int d, const float* pooled, const float* oc,
-                                   const float* doc, float* dpooled, float* stats,
-                                   cudaStream_t s) {
-  static unsigned long long rows_set = 0, cols_set = 0;
-  const int most = static_cast<int>(coarse_backward_smem_bytes(kMaxCubes, 128));
-  cudaError_t err = smem_limit_once(coarse_bwd_rows, most, &rows_set);
-  if (err != cudaSuccess) return err;
-  err = smem_limit_once(coarse_bwd_cols, most, &cols_set);
-  if (err != cudaSuccess) return err;
+                                   const float* doc, float* dpooled, void* workspace,
+                                   size_t workspace_bytes, cudaStream_t s) {
+  const int ldc = coarse_backward_ldc(C);
+  const size_t per = coarse_backward_plane_bytes(C);
+  const long long fit = static_cast<long long>(workspace_bytes / per);
+  const int chunk = static_cast<int>(fit < BH ? fit : BH);
+  if (chunk < 1) return cudaErrorInvalidValue;
   const long long plane = static_cast<long long>(BH) * C * d;
-  const float* qb = pooled;
-  const float* kb = pooled + plane;
-  const float* vb = pooled + 2 * plane;
-  float* row_max = stats;
-  float* row_rz = stats + static_cast<long long>(BH) * C;
-  float* row_D = stats + 2 * static_cast<long long>(BH) * C;
-  const dim3 grid(C, BH);
-  const size_t rows_smem = static_cast<size_t>(2 * d + C) * sizeof(float);
-  coarse_bwd_rows<<<grid, kThreads, rows_smem, s>>>(C, d, qb, kb, vb, oc, doc, dpooled, row_max,
-                                                    row_rz, row_D);
-  err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-  coarse_bwd_cols<<<grid, kThreads, coarse_backward_smem_bytes(C, d), s>>>(
-      C, d, qb, kb, vb, doc, row_max, row_rz, row_D, dpooled + plane, dpooled + 2 * plane);
-  return cudaGetLastError();
+  for (int b0 = 0; b0 < BH; b0 += chunk) {
+    const int nbh = BH - b0 < chunk ? BH - b0 : chunk;
+    const long long off = static_cast<long long>(b0) * C * d;
+    float* sbuf = static_cast<float*>(workspace);
+    float* dpbuf = sbuf + static_cast<long long>(nbh) * C * ldc;
+    const float* qb = pooled + off;
+    const float* kb = pooled + plane + off;
+    const float* vb = pooled + 2 * plane + off;
+    float* dq = dpooled + off;
+    float* dk = dpooled + plane + off;
+    float* dv = dpooled + 2 * plane + off;
+    cudaError_t err =
+        d == 64 ? run_chunk<64>(nbh, C, ldc, qb, kb, vb, oc + off, doc + off, dq, dk, dv, sbuf, dpbuf, s)
+                : run_chunk<128>(nbh, C, ldc, qb, kb, vb, oc + off, doc + off, dq, dk, dv, sbuf, dpbuf, s);
+    if (err != cudaSuccess) return err;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace vsa

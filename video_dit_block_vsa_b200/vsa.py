@@ -36,7 +36,8 @@ EXPORTED = ("vsa_num_cubes", "vsa_topk_from_ratio", "vsa_workspace_bytes", "vsa_
             "vsa_coarse_select_pooled", "vsa_coarse_select_noalloc",
             "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_out",
             "vsa_combine", "vsa_untile", "vsa_forward_host_workspace_bytes", "vsa_forward_host",
-            "vsa_select_transpose", "vsa_backward_prep", "vsa_coarse_backward", "vsa_get_status", "vsa_debug_wait_timeout",
+            "vsa_select_transpose", "vsa_backward_prep", "vsa_coarse_backward_workspace_bytes", "vsa_coarse_backward",
+            "vsa_get_status", "vsa_debug_wait_timeout",
             "vsa_strerror")
 
 
@@ -76,6 +77,7 @@ _sig = {
                                         ctypes.c_int, _P]),
     "vsa_select_transpose": (ctypes.c_int, [_SP, _P, ctypes.c_int, _P, _P, _P, ctypes.c_size_t, _P]),
     "vsa_backward_prep": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+    "vsa_coarse_backward_workspace_bytes": (ctypes.c_size_t, [_SP]),
     "vsa_coarse_backward": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "vsa_get_status": (ctypes.c_int, [_P]),
     "vsa_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
@@ -375,6 +377,10 @@ def vsa_backward_prep(shape, dout, o_fine_tiled, do_fine_tiled, delta, o_coarse=
                                   _ptr(g_fine), _ptr(g_coarse), _ptr(do_fine_tiled), _ptr(delta),
                                   _ptr(do_coarse), _ptr(dg_fine), _ptr(dg_coarse), _stream(stream)),
            "vsa_backward_prep")
+
+
+def vsa_coarse_backward_workspace_bytes(shape) -> int:
+    return int(_lib.vsa_coarse_backward_workspace_bytes(ctypes.byref(shape)))
 
 
 def vsa_coarse_backward(shape, pooled, o_coarse, do_coarse, d_pooled, workspace, stream=None):
