@@ -309,6 +309,33 @@ int vsa_coarse_backward(const vsa_shape* shape, const float* pooled, const float
                         const float* do_coarse, float* d_pooled, void* workspace,
                         size_t workspace_bytes, cudaStream_t stream);
 
+/* Backward of the fine block-sparse attention with the selection held fixed
+ * (the pages describe no backward; this differentiates vsa_block_sparse_fwd
+ * exactly), plus the last steps of the whole backward: the gradient of the
+ * cube means reaches every valid token of its cube, and dq, dk, dv are
+ * written in token order.  With scale = 1/sqrt(d), per query cube i and
+ * selected key cube j: P = exp(scale Q_i K_j^T - lse_i) (0 on pad rows and
+ * keys), dS = P (dO_i V_j^T - delta_i), dQ_i += scale dS K_j,
+ * dK_j += scale dS^T Q_i, dV_j += P^T dO_i; then for a valid row r of cube c
+ * dq[token(r)] = dQ[r] + dqbar[c] / n_c (k and v alike).
+ *   q/k/v_tiled   bf16 [B, H, 64*C, d], the forward's tiled inputs
+ *   sel_idx       int32 [B, H, C, k], the forward's selection
+ *   key_offsets, query_lists  the selection's transpose (vsa_select_transpose)
+ *   lse           float32 [B, H, 64*C] from vsa_block_sparse_fwd
+ *   do_fine_tiled, delta  from vsa_backward_prep
+ *   d_pooled      float32 [3, B, H, C, d] from vsa_coarse_backward, or NULL
+ *                 (ungated: the coarse output does not reach the result)
+ *   dq, dk, dv    bf16 [B, H, N, d] token order (written, every token)
+ * No atomics: one CTA per query cube accumulates dq over its key cubes, one
+ * CTA per key cube accumulates dk, dv over the query cubes that selected it,
+ * so the result is deterministic.  An index outside [0, C) in sel_idx or
+ * query_lists is recorded as VSA_ERR_BAD_INDEX and skipped. */
+int vsa_block_sparse_bwd(const vsa_shape* shape, const void* q_tiled, const void* k_tiled,
+                         const void* v_tiled, const int32_t* sel_idx, int topk,
+                         const int32_t* key_offsets, const int32_t* query_lists, const float* lse,
+                         const void* do_fine_tiled, const float* delta, const float* d_pooled,
+                         void* dq, void* dk, void* dv, cudaStream_t stream);
+
 /* Synchronises `stream`, then returns and clears the status word of the
  * current device: VSA_OK, VSA_ERR_TIMEOUT or VSA_ERR_BAD_INDEX recorded by a
  * kernel since the last call, or VSA_ERR_CUDA if the synchronisation failed. */

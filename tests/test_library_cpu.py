@@ -129,6 +129,13 @@ def test_null_and_misaligned_pointers_rejected_before_launch(vsa):
     assert vsa.vsa_coarse_backward_workspace_bytes(s) == 2 * (2 * 4 * 64 * 4)
     big = vsa.make_shape(1, 40, 128, (21, 45, 80))  # C = 1440, row stride 1472
     assert vsa.vsa_coarse_backward_workspace_bytes(big) == 40 * 2 * 1440 * 1472 * 4
+    fb = lib.vsa_block_sparse_bwd
+    two = ctypes.c_void_p(0x1002)
+    assert fb(ctypes.byref(s), p, p, p, p, 5, p, p, p, p, p, None, p, p, p, None) == vsa.VSA_ERR_INVALID_ARG
+    assert fb(ctypes.byref(s), p, p, p, p, 2, p, p, p, p, p, None, None, p, p, None) == vsa.VSA_ERR_INVALID_ARG
+    assert fb(ctypes.byref(s), odd, p, p, p, 2, p, p, p, p, p, None, p, p, p, None) == vsa.VSA_ERR_INVALID_ARG
+    assert fb(ctypes.byref(s), p, p, p, p, 2, p, p, two, p, p, None, p, p, p, None) == vsa.VSA_ERR_INVALID_ARG
+    assert fb(ctypes.byref(s), p, p, p, p, 2, p, p, p, p, p, odd, p, p, p, None) == vsa.VSA_ERR_INVALID_ARG
     assert lib.vsa_debug_wait_timeout(10, None) == vsa.VSA_ERR_INVALID_ARG
 
 

@@ -35,6 +35,10 @@ cudaError_t launch_backward_prep(const Geom&, const void*, const void*, const fl
 cudaError_t launch_coarse_backward(int, int, int, const float*, const float*, const float*, float*,
                                    void*, size_t, cudaStream_t);
 size_t coarse_backward_plane_bytes(int C);
+cudaError_t launch_block_sparse_bwd(const Geom&, int, const void*, const void*, const void*,
+                                    const void*, const float*, const float*, const int32_t*,
+                                    const int32_t*, const int32_t*, const float*, void*, void*,
+                                    void*, int*, cudaStream_t);
 
 // Device-side status word, one per device that loads the library.
 __device__ int g_status;
@@ -428,6 +432,32 @@ int vsa_coarse_backward(const vsa_shape* shape, const float* pooled, const float
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_coarse_backward(static_cast<int>(bh), g.C, g.d, pooled, o_coarse, do_coarse,
                                         d_pooled, workspace, workspace_bytes, stream));
+}
+
+int vsa_block_sparse_bwd(const vsa_shape* shape, const void* q_tiled, const void* k_tiled,
+                         const void* v_tiled, const int32_t* sel_idx, int topk,
+                         const int32_t* key_offsets, const int32_t* query_lists, const float* lse,
+                         const void* do_fine_tiled, const float* delta, const float* d_pooled,
+                         void* dq, void* dk, void* dv, cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (topk < 1 || topk > g.C) return VSA_ERR_INVALID_ARG;
+  if (!q_tiled || !k_tiled || !v_tiled || !sel_idx || !key_offsets || !query_lists || !lse ||
+      !do_fine_tiled || !delta || !dq || !dk || !dv)
+    return VSA_ERR_INVALID_ARG;
+  auto a4 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; };
+  if (!aligned16(q_tiled) || !aligned16(k_tiled) || !aligned16(v_tiled) ||
+      !aligned16(do_fine_tiled) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (d_pooled && !aligned16(d_pooled)) || !a4(sel_idx) || !a4(key_offsets) ||
+      !a4(query_lists) || !a4(lse) || !a4(delta))
+    return VSA_ERR_INVALID_ARG;
+  if (static_cast<long long>(g.B) * g.H > 65535) return VSA_ERR_UNSUPPORTED;  // grid y
+  DeviceState* st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  return cuda_rc(launch_block_sparse_bwd(g, topk, q_tiled, k_tiled, v_tiled, do_fine_tiled, lse,
+                                         delta, sel_idx, key_offsets, query_lists, d_pooled, dq,
+                                         dk, dv, st->status, stream));
 }
 
 int vsa_get_status(cudaStream_t stream) {

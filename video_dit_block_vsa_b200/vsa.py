@@ -37,7 +37,7 @@ EXPORTED = ("vsa_num_cubes", "vsa_topk_from_ratio", "vsa_workspace_bytes", "vsa_
             "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_out",
             "vsa_combine", "vsa_untile", "vsa_forward_host_workspace_bytes", "vsa_forward_host",
             "vsa_select_transpose", "vsa_backward_prep", "vsa_coarse_backward_workspace_bytes", "vsa_coarse_backward",
-            "vsa_get_status", "vsa_debug_wait_timeout",
+            "vsa_block_sparse_bwd", "vsa_get_status", "vsa_debug_wait_timeout",
             "vsa_strerror")
 
 
@@ -79,6 +79,8 @@ _sig = {
     "vsa_backward_prep": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "vsa_coarse_backward_workspace_bytes": (ctypes.c_size_t, [_SP]),
     "vsa_coarse_backward": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "vsa_block_sparse_bwd": (ctypes.c_int, [_SP, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P, _P, _P,
+                                            _P, _P, _P, _P, _P]),
     "vsa_get_status": (ctypes.c_int, [_P]),
     "vsa_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _P]),
     "vsa_strerror": (ctypes.c_char_p, [ctypes.c_int]),
@@ -396,6 +398,28 @@ def vsa_coarse_backward(shape, pooled, o_coarse, do_coarse, d_pooled, workspace,
            "vsa_coarse_backward")
 
 
+def vsa_block_sparse_bwd(shape, q_tiled, k_tiled, v_tiled, sel_idx, topk, key_offsets, query_lists,
+                         lse, do_fine_tiled, delta, dq, dk, dv, d_pooled=None, stream=None):
+    """Fine-stage backward, pooling backward and untile: dq, dk, dv in token order (see vsa.h)."""
+    B, H, N, d, C = _dims(shape)
+    for n, t in (("q_tiled", q_tiled), ("k_tiled", k_tiled), ("v_tiled", v_tiled),
+                 ("do_fine_tiled", do_fine_tiled)):
+        _expect(t, torch.bfloat16, (B, H, 64 * C, d), n)
+    for n, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _expect(t, torch.bfloat16, (B, H, N, d), n)
+    _expect(sel_idx, torch.int32, (B, H, C, topk), "sel_idx")
+    _expect(key_offsets, torch.int32, (B, H, C + 1), "key_offsets")
+    _expect(query_lists, torch.int32, (B, H, C * topk), "query_lists")
+    _expect(lse, torch.float32, (B, H, 64 * C), "lse")
+    _expect(delta, torch.float32, (B, H, 64 * C), "delta")
+    if d_pooled is not None:
+        _expect(d_pooled, torch.float32, (3, B, H, C, d), "d_pooled")
+    _check(_lib.vsa_block_sparse_bwd(ctypes.byref(shape), _ptr(q_tiled), _ptr(k_tiled), _ptr(v_tiled),
+                                     _ptr(sel_idx), topk, _ptr(key_offsets), _ptr(query_lists), _ptr(lse),
+                                     _ptr(do_fine_tiled), _ptr(delta), _ptr(d_pooled), _ptr(dq), _ptr(dk),
+                                     _ptr(dv), _stream(stream)), "vsa_block_sparse_bwd")
+
+
 def pooled_view(shape, workspace):
     """The pooled qbar, kbar, vbar [3, B, H, C, d] float32 at the start of a
     vsa_tile_permute_pool / vsa_coarse_select workspace (a view, no copy)."""
@@ -454,3 +478,45 @@ def vsa_forward(shape, q, k, v, topk, out, g_fine=None, g_coarse=None, bufs=None
     else:
         vsa_untile(shape, bufs.o_f, out, stream)
     return bufs
+
+
+class VsaGradBuffers:
+    """Device scratch of one backward call, allocated once with torch."""
+
+    def __init__(self, shape: VsaShape, topk: int, gated: bool, device="cuda"):
+        B, H, N, d, C = _dims(shape)
+        f32 = dict(dtype=torch.float32, device=device)
+        self.do_f = torch.empty(B, H, 64 * C, d, dtype=torch.bfloat16, device=device)
+        self.delta = torch.empty(B, H, 64 * C, **f32)
+        self.key_offsets = torch.empty(B, H, C + 1, dtype=torch.int32, device=device)
+        self.query_lists = torch.empty(B, H, C * topk, dtype=torch.int32, device=device)
+        self.transpose_ws = torch.empty(B * H * C * topk * 4, dtype=torch.uint8, device=device)
+        self.do_c = torch.empty(B, H, C, d, **f32) if gated else None
+        self.d_pooled = torch.empty(3, B, H, C, d, **f32) if gated else None
+        self.coarse_ws = (torch.empty(vsa_coarse_backward_workspace_bytes(shape), dtype=torch.uint8,
+                                      device=device) if gated else None)
+
+
+def vsa_backward(shape, bufs, dout, dq, dk, dv, g_fine=None, g_coarse=None, dg_fine=None,
+                 dg_coarse=None, grads=None, stream=None):
+    """Gradients of the whole path for the forward ``bufs`` left (a
+    ``vsa_forward`` with ``VsaBuffers(..., want_lse=True)``): dq, dk, dv
+    ([B, H, N, d] bf16) and, when gated, dg_fine, dg_coarse ([B, H, N] float32).
+    Four library calls: the combine gradient, the coarse backward (gated only),
+    the selection transpose and the fine backward.  Returns the scratch."""
+    if bufs.lse is None:
+        raise ValueError("the forward must keep its LSE (VsaBuffers(..., want_lse=True))")
+    gated = g_fine is not None
+    if grads is None:
+        grads = VsaGradBuffers(shape, bufs.topk, gated, device=dout.device)
+    vsa_backward_prep(shape, dout, bufs.o_f, grads.do_f, grads.delta, bufs.o_c if gated else None,
+                      g_fine, g_coarse, grads.do_c, dg_fine, dg_coarse, stream)
+    if gated:
+        vsa_coarse_backward(shape, pooled_view(shape, bufs.workspace), bufs.o_c, grads.do_c,
+                            grads.d_pooled, grads.coarse_ws, stream)
+    vsa_select_transpose(shape, bufs.sel, bufs.topk, grads.key_offsets, grads.query_lists,
+                         grads.transpose_ws, stream)
+    vsa_block_sparse_bwd(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.sel, bufs.topk, grads.key_offsets,
+                         grads.query_lists, bufs.lse, grads.do_f, grads.delta, dq, dk, dv,
+                         grads.d_pooled if gated else None, stream)
+    return grads
