@@ -120,6 +120,14 @@ def _check(rc: int, where: str):
         raise VsaError(rc, where)
 
 
+def _expect_device(t, name):
+    """A caller-supplied device buffer (workspace): a CUDA tensor."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+
+
 def _expect(t, dtype, shape, name):
     if t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
@@ -180,6 +188,7 @@ def vsa_coarse_select(shape, q_tiled, k_tiled, v_tiled, cube_count, topk, sel_id
         _expect(o_coarse, torch.float32, (B, H, C, d), "o_coarse")
     if coarse_logits is not None:
         _expect(coarse_logits, torch.float32, (B, H, C, C), "coarse_logits")
+    _expect_device(workspace, "workspace")
     _check(_lib.vsa_coarse_select(ctypes.byref(shape), _ptr(q_tiled), _ptr(k_tiled), _ptr(v_tiled),
                                   _ptr(cube_count), topk, _ptr(o_coarse), _ptr(sel_idx),
                                   _ptr(coarse_logits), _ptr(workspace),
@@ -198,6 +207,7 @@ def vsa_coarse_select_tokens(shape, q, k, v, topk, sel_idx, workspace, o_coarse=
         _expect(o_coarse, torch.float32, (B, H, C, d), "o_coarse")
     if coarse_logits is not None:
         _expect(coarse_logits, torch.float32, (B, H, C, C), "coarse_logits")
+    _expect_device(workspace, "workspace")
     _check(_lib.vsa_coarse_select_tokens(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), topk,
                                          _ptr(o_coarse), _ptr(sel_idx), _ptr(coarse_logits),
                                          _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -214,6 +224,7 @@ def vsa_tile_permute_pool(shape, q, k, v, q_tiled, k_tiled, v_tiled, workspace, 
         _expect(t, torch.bfloat16, (B, H, 64 * C, d), n)
     if cube_count is not None:
         _expect(cube_count, torch.int32, (C,), "cube_count")
+    _expect_device(workspace, "workspace")
     _check(_lib.vsa_tile_permute_pool(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(q_tiled),
                                       _ptr(k_tiled), _ptr(v_tiled), _ptr(cube_count), _ptr(workspace),
                                       workspace.numel() * workspace.element_size(), _stream(stream)),
@@ -229,6 +240,7 @@ def vsa_coarse_select_pooled(shape, topk, sel_idx, workspace, o_coarse=None, coa
         _expect(o_coarse, torch.float32, (B, H, C, d), "o_coarse")
     if coarse_logits is not None:
         _expect(coarse_logits, torch.float32, (B, H, C, C), "coarse_logits")
+    _expect_device(workspace, "workspace")
     _check(_lib.vsa_coarse_select_pooled(ctypes.byref(shape), topk, _ptr(o_coarse), _ptr(sel_idx),
                                          _ptr(coarse_logits), _ptr(workspace),
                                          workspace.numel() * workspace.element_size(), _stream(stream)),
@@ -356,6 +368,7 @@ def vsa_select_transpose(shape, sel_idx, topk, key_offsets, query_lists, workspa
     _expect(sel_idx, torch.int32, (B, H, C, topk), "sel_idx")
     _expect(key_offsets, torch.int32, (B, H, C + 1), "key_offsets")
     _expect(query_lists, torch.int32, (B, H, C * topk), "query_lists")
+    _expect_device(workspace, "workspace")
     _check(_lib.vsa_select_transpose(ctypes.byref(shape), _ptr(sel_idx), topk, _ptr(key_offsets),
                                      _ptr(query_lists), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream(stream)),
@@ -392,6 +405,7 @@ def vsa_coarse_backward(shape, pooled, o_coarse, do_coarse, d_pooled, workspace,
     _expect(o_coarse, torch.float32, (B, H, C, d), "o_coarse")
     _expect(do_coarse, torch.float32, (B, H, C, d), "do_coarse")
     _expect(d_pooled, torch.float32, (3, B, H, C, d), "d_pooled")
+    _expect_device(workspace, "workspace")
     _check(_lib.vsa_coarse_backward(ctypes.byref(shape), _ptr(pooled), _ptr(o_coarse), _ptr(do_coarse),
                                     _ptr(d_pooled), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream(stream)),
