@@ -206,6 +206,10 @@ int main(void) {
   if (vsa_workspace_bytes(&s, k) != (size_t)3 * 40 * 1440 * 128 * 4) return 3;
   if (strcmp(vsa_strerror(VSA_OK), "ok") != 0) return 4;
   if (vsa_tile_permute(&s, NULL, NULL, NULL, 0) != VSA_ERR_INVALID_ARG) return 5;
+  /* two C x C float32 matrices per (b, h), rows padded to 1472 */
+  if (vsa_coarse_backward_workspace_bytes(&s) != (size_t)40 * 2 * 1440 * 1472 * 4) return 6;
+  if (vsa_block_sparse_bwd(&s, NULL, NULL, NULL, NULL, k, NULL, NULL, NULL, NULL, NULL, NULL,
+                           NULL, NULL, NULL, 0) != VSA_ERR_INVALID_ARG) return 7;
   printf("c abi ok\n");
   return 0;
 }
