@@ -171,18 +171,21 @@ def combine_backward(dout_t, of_t, oc, counts, grid, g_f=None, g_c=None, cube=CU
     return dof, doc, dgf, dgc
 
 
-def vsa_backward(q, k, v, grid, topk, dout, g_f=None, g_c=None, cube=CUBE):
+def vsa_backward(q, k, v, grid, topk, dout, g_f=None, g_c=None, cube=CUBE, sel=None):
     """Gradients of <dout, out> for the whole path on float64 arrays [B, Hh, N, d].
 
-    Returns dict(dq, dk, dv [B, Hh, N, d], dg_f, dg_c [B, Hh, N] or None, sel)
-    with the selection held at the forward's choice.
+    Returns dict(dq, dk, dv [B, Hh, N, d], dg_f, dg_c [B, Hh, N] or None, sel,
+    S_c) with the selection held at the forward's choice.  ``sel`` replaces
+    that choice with another valid one (a top-k set of S_c up to ties); the
+    arithmetic is the same.
     """
     q_t, counts = tile_permute(q, grid, cube)
     k_t, _ = tile_permute(k, grid, cube)
     v_t, _ = tile_permute(v, grid, cube)
     qb, kb, vb = pool(q_t, counts), pool(k_t, counts), pool(v_t, counts)
     S_c, O_c = coarse_attention(qb, kb, vb)
-    sel = topk_select(S_c, topk)
+    if sel is None:
+        sel = topk_select(S_c, topk)
     O_f, _ = block_sparse_attention(q_t, k_t, v_t, counts, sel)
     dout_t, _ = tile_permute(dout, grid, cube)
     dof, doc, dgf, dgc = combine_backward(dout_t, O_f, O_c, counts, grid, g_f, g_c, cube)
@@ -193,7 +196,7 @@ def vsa_backward(q, k, v, grid, topk, dout, g_f=None, g_c=None, cube=CUBE):
     dk_t += pool_backward(dkb, counts, S)
     dv_t += pool_backward(dvb, counts, S)
     return dict(dq=untile(dq_t, grid, cube), dk=untile(dk_t, grid, cube),
-                dv=untile(dv_t, grid, cube), dg_f=dgf, dg_c=dgc, sel=sel)
+                dv=untile(dv_t, grid, cube), dg_f=dgf, dg_c=dgc, sel=sel, S_c=S_c)
 
 
 __all__ = ["attention_backward", "attention_backward_from_lse", "select_transpose",

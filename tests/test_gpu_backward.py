@@ -21,7 +21,7 @@ import torch
 from oracle import vsa_backward as vb
 from oracle import vsa_oracle as vo
 from video_dit_block_vsa_b200 import workloads as wl
-from tests.vsa_checks import bf16_dev_to_f64, to_dev_bf16
+from tests.vsa_checks import bf16_dev_to_f64, check_selection, to_dev_bf16
 
 pytestmark = [
     pytest.mark.gpu,
@@ -87,9 +87,12 @@ def test_backward_matches_oracle(vsa, w, heads):
     f64 = lambda n: vo.bf16_bits_to_f64(x[n])
     gf = x["g_f"].astype(np.float64) if w.gated else None
     gc = x["g_c"].astype(np.float64) if w.gated else None
-    ref = vb.vsa_backward(f64("q"), f64("k"), f64("v"), w.grid, w.topk,
-                          vo.bf16_bits_to_f64(dout_bits), gf, gc)
-    assert np.array_equal(bufs.sel.cpu().numpy(), ref["sel"]), "selection differs from the oracle"
+    args = (f64("q"), f64("k"), f64("v"), w.grid, w.topk, vo.bf16_bits_to_f64(dout_bits), gf, gc)
+    ref = vb.vsa_backward(*args)
+    sel = bufs.sel.cpu().numpy().astype(np.int64)
+    equal, swapped = check_selection(sel, ref["S_c"], w.topk)  # a top-k set up to the tie band
+    if swapped:  # gradients of the GPU's (equally valid) selection
+        ref = vb.vsa_backward(*args, sel=sel)
     check(bf16_dev_to_f64(dq), ref["dq"], "dq")
     check(bf16_dev_to_f64(dk), ref["dk"], "dk")
     check(bf16_dev_to_f64(dv), ref["dv"], "dv")
