@@ -303,8 +303,11 @@ def run_gpu(args, w):
     # "block_sparse_fwd" is the fine kernel with the combine and untile steps
     # in its epilogue
     pairs = {"tile_permute": (0, 1), "coarse_select": (1, 2), "block_sparse_fwd": (2, 3)}
-    stage_ms = {name: statistics.mean(evs[s][a_].elapsed_time(evs[s][b_]) for s in range(args.steps))
-                for name, (a_, b_) in pairs.items()}
+    stage_all = {name: [evs[s][a_].elapsed_time(evs[s][b_]) for s in range(args.steps)]
+                 for name, (a_, b_) in pairs.items()}
+    stage_ms = {name: statistics.mean(v_) for name, v_ in stage_all.items()}
+    step_all = [evs[s][0].elapsed_time(evs[s][3]) for s in range(args.steps)]
+    spread = lambda v_: {"mean": statistics.mean(v_), "median": statistics.median(v_), "min": min(v_)}
     ms_per_step = elapsed_ms / args.steps
     value = vdist.job_throughput(step_flops, args.steps, elapsed_ms, world) / 1e12
 
@@ -363,10 +366,16 @@ def run_gpu(args, w):
             "achieved": kv_bytes / (fine_ms * 1e-3) / 1e12, "peak": feed_peak, "unit": "TB/s",
             "frac": kv_bytes / (fine_ms * 1e-3) / 1e12 / feed_peak,
             "peak_kind": f"{TMA_INGEST_GBS_PER_SM} GB/s per SM (measured) x {sms} SMs"}
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_sustained"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_sustained"], "traffic": traffic,
-                "kernel": "vsa_block_sparse_fwd_out (fine attention; combine and untile in its epilogue)", "peak_kind": f"bf16 sustained ({peaks['source']})",
-                "peak_burst": peaks["bf16"], "frac_of_burst": achieved / peaks["bf16"],
+    # The fine kernel runs for tens of milliseconds inside a step of the same
+    # length, so its denominator is the burst bf16 figure; the sustained
+    # (seconds-long, power-capped) figure is reported beside it.
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16"], "traffic": traffic,
+                "kernel": "vsa_block_sparse_fwd_out (fine attention; combine and untile in its epilogue)",
+                "peak_kind": f"bf16 burst ({peaks['source']})",
+                "peak_sustained": peaks["bf16_sustained"],
+                "frac_of_sustained": achieved / peaks["bf16_sustained"],
+                "kernel_ms": spread(stage_all["block_sparse_fwd"]),
                 "issued_tflops": fine_issued / (fine_ms * 1e-3) / 1e12, "feed": feed}
 
     cpu = None
@@ -400,6 +409,7 @@ def run_gpu(args, w):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clk,
             "stages_ms": stage_ms,
+            "step_ms": spread(step_all),
             "stages_note": ("tile_permute is one pass that tiles q, k, v and writes their cube "
                             "means (the coarse stage's pooling); coarse_select starts from those; "
                             "block_sparse_fwd writes the final token-order output, applying the "

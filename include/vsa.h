@@ -32,8 +32,13 @@
  *     successful launch; argument errors are reported before any launch and
  *     nothing is written.
  *   - Device-side conditions (a bounded wait that ran out, an inconsistent
- *     cube_count / sel_idx entry) are recorded in a per-device status word
- *     read and cleared by vsa_get_status().  Kernels never trap.
+ *     cube_count / sel_idx entry) are recorded in a status word of the
+ *     current CUDA context, read and cleared by vsa_get_status().  Kernels
+ *     never trap.
+ *   - Calls work in whatever CUDA context is current on the calling thread
+ *     (the device's primary context by default); values the library keeps
+ *     per context (the status word's address, raised kernel limits, the host
+ *     path's copy streams) are looked up again in a new context.
  *   - Calls on one device from several host threads are safe; calls that
  *     overlap on the GPU and write the same output race, as any CUDA kernel.
  */
@@ -160,8 +165,10 @@ int vsa_coarse_select_tokens(const vsa_shape* shape, const void* q, const void* 
  *     before any launch; use vsa_coarse_select with a workspace for them.
  *   - Every GPU context that loads the library holds the 32 MiB from module
  *     load until the process exits.
- *   - The first call on a device looks up the array's device address (with
- *     that device current); make that first call before any stream capture.
+ *   - The first call in each CUDA context (the device's primary context, a
+ *     context the caller made current, or the new primary context after
+ *     cudaDeviceReset) looks up the array's device address in that context;
+ *     make that first call before any stream capture.
  *   - All calls on a device share the one array: calls that overlap on the
  *     GPU (different streams, no ordering between them) race on it.  Calls
  *     ordered on one stream are safe.  The array keeps the last call's

@@ -9,10 +9,7 @@ lands within 4e-3 (max) and 2.4e-4 (mean) of the largest gradient on these
 cases; the bounds below leave 2.5x and 4x of room.  A wrong index, a
 transposed operand or a dropped term is off by the gradient's own size.
 
-These kernels have not run on a B200 yet: the tests run only with
-VSA_RUN_FINE_BACKWARD_TESTS=1."""
-
-import os
+"""
 
 import numpy as np
 import pytest
@@ -23,12 +20,7 @@ from oracle import vsa_oracle as vo
 from video_dit_block_vsa_b200 import workloads as wl
 from tests.vsa_checks import bf16_dev_to_f64, check_selection, to_dev_bf16
 
-pytestmark = [
-    pytest.mark.gpu,
-    pytest.mark.skipif(os.environ.get("VSA_RUN_FINE_BACKWARD_TESTS") != "1",
-                       reason="fine backward kernels not yet run on a B200; "
-                              "set VSA_RUN_FINE_BACKWARD_TESTS=1"),
-]
+pytestmark = pytest.mark.gpu
 
 MAX_REL = 1e-2   # max |got - ref| / max |ref|, per gradient
 MEAN_REL = 1e-3  # mean |got - ref| / max |ref|

@@ -341,32 +341,56 @@ def sampled_cubes(counts, n, seed):
 
 
 def check_workload(vsa, w, head_sample=None, cube_sample=None):
+    """Runs the workload through both forms of the public forward call and
+    checks them against the oracle:
+      - the three launches the benchmark times (``vsa_forward_fused``: tiling
+        with pooling, coarse stage from the means, fine kernel writing the gated
+        token-order output), on every head: tiled q, k, v bit-exact, selection
+        tie-aware; the output on the sampled heads and query cubes;
+      - the five separate calls (``vsa_forward``): selection and output
+        bit-identical to the fused form on every head."""
     x = wl.make_inputs(w)
     shape = vsa.make_shape(w.batch, w.heads, w.head_dim, w.grid)
     q, k, v = (to_dev_bf16(x[n]) for n in ("q", "k", "v"))
     g_f = torch.from_numpy(x["g_f"]).cuda() if w.gated else None
     g_c = torch.from_numpy(x["g_c"]).cuda() if w.gated else None
     out = torch.empty_like(q)
-    bufs = vsa.vsa_forward(shape, q, k, v, w.topk, out, g_f, g_c)
+    bufs = vsa.vsa_forward_fused(shape, q, k, v, w.topk, out, g_f, g_c)
     torch.cuda.synchronize()
     assert vsa.vsa_get_status() == 0
+    # the separate calls: same selection and output bits as the fused form
+    out_calls = torch.empty_like(q)
+    bufs_calls = vsa.vsa_forward(shape, q, k, v, w.topk, out_calls, g_f, g_c)
+    torch.cuda.synchronize()
+    assert vsa.vsa_get_status() == 0
+    assert torch.equal(bufs_calls.sel, bufs.sel), f"{w.name}: selections of the two forms differ"
+    assert torch.equal(out_calls.view(torch.int16), out.view(torch.int16)), \
+        f"{w.name}: outputs of the two forms differ"
+    del bufs_calls, out_calls
     sel_gpu = bufs.sel.cpu().numpy()
     heads = [(b, h) for b in range(w.batch) for h in range(w.heads)]
+    sampled = set(heads)
     if head_sample is not None:
         rng = np.random.default_rng(w.seed)
         idx = sorted(rng.choice(len(heads), head_sample, replace=False).tolist())
-        heads = [heads[i] for i in idx]
+        sampled = {heads[i] for i in idx}
     slot_token, counts = vo.cube_permutation(w.grid)
+    assert np.array_equal(bufs.counts.cpu().numpy(), counts)
     for b, h in heads:
-        one = lambda n: vo.bf16_bits_to_f64(x[n][b:b + 1, h:h + 1])
-        gf = x["g_f"][b:b + 1, h:h + 1].astype(np.float64) if w.gated else None
-        gc = x["g_c"][b:b + 1, h:h + 1].astype(np.float64) if w.gated else None
-        q_t, _ = vo.tile_permute(one("q"), w.grid)
-        k_t, _ = vo.tile_permute(one("k"), w.grid)
-        v_t, _ = vo.tile_permute(one("v"), w.grid)
+        tiled = {}
+        for n, dev_t in (("q", bufs.q_t), ("k", bufs.k_t), ("v", bufs.v_t)):
+            ref_bits, _ = vo.tile_permute(x[n][b:b + 1, h:h + 1], w.grid)
+            assert np.array_equal(bf16_dev_bits(dev_t[b, h]), ref_bits[0, 0]), \
+                f"{w.name}: tiled {n} differs (b={b}, h={h})"
+            tiled[n] = vo.bf16_bits_to_f64(ref_bits)
+        q_t, k_t, v_t = tiled["q"], tiled["k"], tiled["v"]
         S, O_c = vo.coarse_attention(vo.pool(q_t, counts), vo.pool(k_t, counts), vo.pool(v_t, counts))
         sel = sel_gpu[b:b + 1, h:h + 1]
         check_selection(sel, S, w.topk)  # selection up to ties; outputs use the GPU's choice
+        if (b, h) not in sampled:
+            continue
+        gf = x["g_f"][b:b + 1, h:h + 1].astype(np.float64) if w.gated else None
+        gc = x["g_c"][b:b + 1, h:h + 1].astype(np.float64) if w.gated else None
         cubes = None if cube_sample is None else sampled_cubes(counts, cube_sample, w.seed + h)
         O_f, _ = vo.block_sparse_attention(q_t, k_t, v_t, counts, sel, query_cubes=cubes)
         ref = vo.untile(vo.combine(O_f, O_c, counts, w.grid, gf, gc), w.grid)[0, 0]

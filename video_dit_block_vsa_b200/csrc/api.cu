@@ -47,15 +47,29 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// What the library needs per call on the current device: hardware facts (the
+// same in every context on the device) and the status word's device address
+// (valid only in the context it was looked up in).
 struct DeviceState {
+  int sms = 0;
+  int* status = nullptr;
+};
+
+struct DeviceInfo {
   bool ready = false;
   int supported = 0;
   int sms = 0;
-  int* status = nullptr;  // device address of g_status
 };
 
 std::mutex g_mu;
-DeviceState g_dev[kMaxDevices];
+DeviceInfo g_dev[kMaxDevices];
+CtxCache<int*> g_status_ptr;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+std::once_flag g_ctx_fns_once;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -63,44 +77,52 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
 
-// Per-device setup on first use: architecture check and the status word's
-// device address (a host-side symbol is not a device pointer).
-int device_state(DeviceState** out) {
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(fn);
+}
+
+// Per-call setup: architecture check (once per device) and the status word's
+// device address in the current context (a host-side symbol is not a device
+// pointer; the address is looked up once per context).
+int device_state(DeviceState* out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return VSA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_mu);
-  DeviceState& st = g_dev[dev];
-  if (!st.ready) {
-    int major = 0, minor = 0, sms = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return VSA_ERR_CUDA;
-    st.supported = (major == 10 && minor == 0);
-    st.sms = sms;
-    if (st.supported) {
-      void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return VSA_ERR_CUDA;
-      st.status = static_cast<int*>(p);
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo& di = g_dev[dev];
+    if (!di.ready) {
+      int major = 0, minor = 0, sms = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return VSA_ERR_CUDA;
+      di.supported = (major == 10 && minor == 0);
+      di.sms = sms;
+      di.ready = true;
     }
-    st.ready = true;
+    if (!di.supported) return VSA_ERR_UNSUPPORTED;
+    out->sms = di.sms;
   }
-  if (!st.supported) return VSA_ERR_UNSUPPORTED;
-  *out = &st;
-  return VSA_OK;
+  const bool ok = g_status_ptr.get(current_context_id(), [](int** p) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_status) != cudaSuccess || a == nullptr) return false;
+    *p = static_cast<int*>(a);
+    return true;
+  }, &out->status);
+  return ok ? VSA_OK : VSA_ERR_CUDA;
 }
 
 int get_encoder() {
   std::lock_guard<std::mutex> lock(g_mu);
   if (g_encode) return VSA_OK;
-  void* fn = nullptr;
-  cudaDriverEntryPointQueryResult q;
-  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
-          cudaSuccess ||
-      q != cudaDriverEntryPointSuccess || fn == nullptr)
-    return VSA_ERR_CUDA;
-  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
-  return VSA_OK;
+  g_encode = driver_fn<EncodeTiledFn>("cuTensorMapEncodeTiled");
+  return g_encode ? VSA_OK : VSA_ERR_CUDA;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -153,6 +175,30 @@ int cuda_rc(cudaError_t e) { return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA; }
 }  // namespace
 }  // namespace vsa
 
+namespace vsa {
+
+uint64_t current_context_id() {
+  std::call_once(g_ctx_fns_once, [] {
+    g_ctx_get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    g_ctx_get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  });
+  if (g_ctx_get_current == nullptr || g_ctx_get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return 0;
+  if (ctx == nullptr) {
+    // No context on this thread yet: make the current device's primary
+    // context current, as the next runtime call would.
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return 0;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  }
+  unsigned long long id = 0;
+  if (g_ctx_get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+}  // namespace vsa
+
 using namespace vsa;
 
 extern "C" {
@@ -191,9 +237,9 @@ int vsa_tile_permute(const vsa_shape* shape, const void* x, void* x_tiled, int32
   if (!x || !x_tiled || !aligned16(x) || !aligned16(x_tiled) ||
       (cube_count && (reinterpret_cast<uintptr_t>(cube_count) & 3u)))
     return VSA_ERR_INVALID_ARG;
-  DeviceState* st;
+  DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
-  return cuda_rc(launch_tile_permute(g, x, x_tiled, cube_count, st->sms, stream));
+  return cuda_rc(launch_tile_permute(g, x, x_tiled, cube_count, st.sms, stream));
 }
 
 int vsa_untile(const vsa_shape* shape, const void* x_tiled, void* x, cudaStream_t stream) {
@@ -201,9 +247,9 @@ int vsa_untile(const vsa_shape* shape, const void* x_tiled, void* x, cudaStream_
   int rc = make_geom(shape, &g);
   if (rc != VSA_OK) return rc;
   if (!x || !x_tiled || !aligned16(x) || !aligned16(x_tiled)) return VSA_ERR_INVALID_ARG;
-  DeviceState* st;
+  DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
-  return cuda_rc(launch_untile(g, x_tiled, x, st->sms, stream));
+  return cuda_rc(launch_untile(g, x_tiled, x, st.sms, stream));
 }
 
 int vsa_combine(const vsa_shape* shape, const void* o_fine_tiled, const float* o_coarse,
@@ -218,9 +264,9 @@ int vsa_combine(const vsa_shape* shape, const void* o_fine_tiled, const float* o
                  (reinterpret_cast<uintptr_t>(g_fine) & 3u) ||
                  (reinterpret_cast<uintptr_t>(g_coarse) & 3u)))
     return VSA_ERR_INVALID_ARG;
-  DeviceState* st;
+  DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
-  return cuda_rc(launch_combine(g, o_fine_tiled, o_coarse, g_fine, g_coarse, out_tiled, st->sms,
+  return cuda_rc(launch_combine(g, o_fine_tiled, o_coarse, g_fine, g_coarse, out_tiled, st.sms,
                                 stream));
 }
 
@@ -241,11 +287,11 @@ int vsa_coarse_select(const vsa_shape* shape, const void* q_tiled, const void* k
       (coarse_logits && (reinterpret_cast<uintptr_t>(coarse_logits) & 3u)))
     return VSA_ERR_INVALID_ARG;
   if (workspace_bytes < vsa_workspace_bytes(shape, topk)) return VSA_ERR_INVALID_ARG;
-  DeviceState* st;
+  DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_coarse_select(g, q_tiled, k_tiled, v_tiled, cube_count, topk, o_coarse,
                                       sel_idx, coarse_logits, static_cast<float*>(workspace),
-                                      st->status, stream, false));
+                                      st.status, stream, false));
 }
 
 int vsa_tile_permute_pool(const vsa_shape* shape, const void* q, const void* k, const void* v,
@@ -261,10 +307,10 @@ int vsa_tile_permute_pool(const vsa_shape* shape, const void* q, const void* k, 
       (cube_count && (reinterpret_cast<uintptr_t>(cube_count) & 3u)))
     return VSA_ERR_INVALID_ARG;
   if (workspace_bytes < vsa_workspace_bytes(shape, 1)) return VSA_ERR_INVALID_ARG;
-  DeviceState* st;
+  DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_tile_pool(g, q, k, v, q_tiled, k_tiled, v_tiled, cube_count,
-                                  static_cast<float*>(workspace), st->status, stream));
+                                  static_cast<float*>(workspace), st.status, stream));
 }
 
 int vsa_coarse_select_pooled(const vsa_shape* shape, int topk, float* o_coarse, int32_t* sel_idx,
@@ -280,7 +326,7 @@ int vsa_coarse_select_pooled(const vsa_shape* shape, int topk, float* o_coarse, 
       (coarse_logits && (reinterpret_cast<uintptr_t>(coarse_logits) & 3u)))
     return VSA_ERR_INVALID_ARG;
   if (workspace_bytes < vsa_workspace_bytes(shape, topk)) return VSA_ERR_INVALID_ARG;
-  DeviceState* st;
+  DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_coarse_only(g, topk, o_coarse, sel_idx, coarse_logits,
                                     static_cast<const float*>(workspace), stream));
@@ -300,10 +346,10 @@ int vsa_coarse_select_tokens(const vsa_shape* shape, const void* q, const void* 
       (coarse_logits && (reinterpret_cast<uintptr_t>(coarse_logits) & 3u)))
     return VSA_ERR_INVALID_ARG;
   if (workspace_bytes < vsa_workspace_bytes(shape, topk)) return VSA_ERR_INVALID_ARG;
-  DeviceState* st;
+  DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_coarse_select(g, q, k, v, nullptr, topk, o_coarse, sel_idx, coarse_logits,
-                                      static_cast<float*>(workspace), st->status, stream, true));
+                                      static_cast<float*>(workspace), st.status, stream, true));
 }
 
 int vsa_block_sparse_fwd(const vsa_shape* shape, const void* q_tiled, const void* k_tiled,
@@ -320,7 +366,7 @@ int vsa_block_sparse_fwd(const vsa_shape* shape, const void* q_tiled, const void
       (reinterpret_cast<uintptr_t>(sel_idx) & 3u) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return VSA_ERR_INVALID_ARG;
-  DeviceState* st;
+  DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   if ((rc = get_encoder()) != VSA_OK) return rc;
   CUtensorMap tq, tk, tv;
@@ -328,7 +374,7 @@ int vsa_block_sparse_fwd(const vsa_shape* shape, const void* q_tiled, const void
       tiled_map(g, v_tiled, &tv) != VSA_OK)
     return VSA_ERR_CUDA;
   return cuda_rc(launch_block_sparse_fwd(g, tq, tk, tv, cube_count, sel_idx, topk, o_fine_tiled,
-                                         lse, nullptr, nullptr, nullptr, false, st->status, st->sms,
+                                         lse, nullptr, nullptr, nullptr, false, st.status, st.sms,
                                          stream));
 }
 
@@ -352,7 +398,7 @@ int vsa_block_sparse_fwd_out(const vsa_shape* shape, const void* q_tiled, const 
       (reinterpret_cast<uintptr_t>(sel_idx) & 3u) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return VSA_ERR_INVALID_ARG;
-  DeviceState* st;
+  DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   if ((rc = get_encoder()) != VSA_OK) return rc;
   CUtensorMap tq, tk, tv;
@@ -361,7 +407,7 @@ int vsa_block_sparse_fwd_out(const vsa_shape* shape, const void* q_tiled, const 
     return VSA_ERR_CUDA;
   return cuda_rc(launch_block_sparse_fwd(g, tq, tk, tv, cube_count, sel_idx, topk, out, lse,
                                          g_fine ? o_coarse : nullptr, g_fine, g_coarse, true,
-                                         st->status, st->sms, stream));
+                                         st.status, st.sms, stream));
 }
 
 int vsa_select_transpose(const vsa_shape* shape, const int32_t* sel_idx, int topk,
@@ -378,10 +424,10 @@ int vsa_select_transpose(const vsa_shape* shape, const int32_t* sel_idx, int top
   const long long pairs = static_cast<long long>(g.B) * g.H * g.C * topk;
   if (static_cast<long long>(g.C) * topk >= (1ll << 31)) return VSA_ERR_UNSUPPORTED;
   if (workspace_bytes < static_cast<size_t>(pairs) * sizeof(int32_t)) return VSA_ERR_INVALID_ARG;
-  DeviceState* st;
+  DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_select_transpose(g.B * g.H, g.C, topk, sel_idx, key_offsets, query_lists,
-                                         static_cast<int32_t*>(workspace), st->status, stream));
+                                         static_cast<int32_t*>(workspace), st.status, stream));
 }
 
 int vsa_backward_prep(const vsa_shape* shape, const void* dout, const void* o_fine_tiled,
@@ -401,7 +447,7 @@ int vsa_backward_prep(const vsa_shape* shape, const void* dout, const void* o_fi
   if (gated && (!aligned16(o_coarse) || !aligned16(do_coarse) || !a4(g_fine) || !a4(g_coarse) ||
                 !a4(dg_fine) || !a4(dg_coarse)))
     return VSA_ERR_INVALID_ARG;
-  DeviceState* st;
+  DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_backward_prep(g, dout, o_fine_tiled, gated ? o_coarse : nullptr,
                                       g_fine, g_coarse, do_fine_tiled, delta,
@@ -428,7 +474,7 @@ int vsa_coarse_backward(const vsa_shape* shape, const float* pooled, const float
   const long long bh = static_cast<long long>(g.B) * g.H;
   if (bh > 65535) return VSA_ERR_UNSUPPORTED;  // (b, h) is a grid index
   if (workspace_bytes < coarse_backward_plane_bytes(g.C)) return VSA_ERR_INVALID_ARG;
-  DeviceState* st;
+  DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_coarse_backward(static_cast<int>(bh), g.C, g.d, pooled, o_coarse, do_coarse,
                                         d_pooled, workspace, workspace_bytes, stream));
@@ -453,32 +499,32 @@ int vsa_block_sparse_bwd(const vsa_shape* shape, const void* q_tiled, const void
       !a4(query_lists) || !a4(lse) || !a4(delta))
     return VSA_ERR_INVALID_ARG;
   if (static_cast<long long>(g.B) * g.H > 65535) return VSA_ERR_UNSUPPORTED;  // grid y
-  DeviceState* st;
+  DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_block_sparse_bwd(g, topk, q_tiled, k_tiled, v_tiled, do_fine_tiled, lse,
                                          delta, sel_idx, key_offsets, query_lists, d_pooled, dq,
-                                         dk, dv, st->status, stream));
+                                         dk, dv, st.status, stream));
 }
 
 int vsa_get_status(cudaStream_t stream) {
-  DeviceState* st;
+  DeviceState st;
   int rc = device_state(&st);
   if (rc != VSA_OK) return rc;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return VSA_ERR_CUDA;
   int value = 0;
   const int zero = 0;
-  if (cudaMemcpy(&value, st->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
-      cudaMemcpy(st->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+  if (cudaMemcpy(&value, st.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(st.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return VSA_ERR_CUDA;
   return value;
 }
 
 int vsa_debug_wait_timeout(uint64_t timeout_ns, cudaStream_t stream) {
   if (timeout_ns < 1000ull || timeout_ns > 1000000000ull) return VSA_ERR_INVALID_ARG;
-  DeviceState* st;
+  DeviceState st;
   const int rc = device_state(&st);
   if (rc != VSA_OK) return rc;
-  return cuda_rc(launch_debug_wait(timeout_ns, st->status, stream));
+  return cuda_rc(launch_debug_wait(timeout_ns, st.status, stream));
 }
 
 const char* vsa_strerror(int code) {

@@ -428,7 +428,7 @@ cudaError_t launch_coarse_only(const Geom& g, int topk, float* o_coarse, int32_t
   // the limit is raised once per device to the largest block any accepted
   // shape needs: the logits block never exceeds kLogitBudgetBytes, plus qT
   // for d = 128, the staging buffer and the top-k histograms
-  static unsigned long long limit_set = 0;
+  static CtxCache<char> limit_set;
   const size_t most = kLogitBudgetBytes + (static_cast<size_t>(128) * 16 + kStageFloats) * sizeof(float) +
                       8 * 256 * sizeof(int);
   err = smem_limit_once(coarse_kernel, static_cast<int>(most), &limit_set);

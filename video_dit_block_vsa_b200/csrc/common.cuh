@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include "ctx_cache.h"
 #include "vsa.h"
 
 namespace vsa {
@@ -73,19 +74,27 @@ __device__ __forceinline__ long long slot_token(const Geom& g, int c, int s) {
   return (static_cast<long long>(t0 + lt) * g.Y + (y0 + ly)) * g.X + (x0 + lx);
 }
 
-// Raises a kernel's dynamic shared-memory limit once per device (bit d of
-// *done for device d), so that later launches, including launches made
-// while a stream is being captured into a CUDA graph, only launch.
+// Unique id of the CUDA context current on this thread; if none is current,
+// the current device's primary context is made current first.  0 if it
+// cannot be determined.  Values cached per context (CtxCache) use it as key.
+uint64_t current_context_id();
+
+// Raises a kernel's dynamic shared-memory limit once per CUDA context, so
+// that later launches, including launches made while a stream is being
+// captured into a CUDA graph, only launch.  The attribute belongs to the
+// context, so a new context (after cudaDeviceReset, or one the caller made
+// current) gets it raised again.
 template <typename Kernel>
-inline cudaError_t smem_limit_once(Kernel kernel, int bytes, unsigned long long* done) {
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
-  const unsigned long long bit = 1ull << (dev & 63);
-  if (__atomic_load_n(done, __ATOMIC_ACQUIRE) & bit) return cudaSuccess;
-  err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (err == cudaSuccess) __atomic_fetch_or(done, bit, __ATOMIC_RELEASE);
-  return err;
+inline cudaError_t smem_limit_once(Kernel kernel, int bytes, CtxCache<char>* done) {
+  cudaError_t err = cudaSuccess;
+  char ok = 0;
+  const bool got = done->get(current_context_id(), [&](char* v) {
+    err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    *v = 1;
+    return err == cudaSuccess;
+  }, &ok);
+  if (got) return cudaSuccess;
+  return err != cudaSuccess ? err : cudaErrorInvalidValue;
 }
 
 // Record a device-side condition in the status word (first one wins).

@@ -594,7 +594,7 @@ cudaError_t launch_block_sparse_fwd(const Geom& g, const CUtensorMap& tq, const 
                    token_order ? 1 : 0};
   cudaError_t err;
   // one kernel per head dim and output form; each raises its smem limit once
-  static unsigned long long limit_set[4] = {0, 0, 0, 0};
+  static CtxCache<char> limit_set[4];
   auto run = [&](auto kernel, int which) -> cudaError_t {
     cudaError_t e = smem_limit_once(kernel, static_cast<int>(smem), &limit_set[which]);
     if (e != cudaSuccess) return e;

@@ -234,7 +234,7 @@ cudaError_t run(const Geom& g, int topk, const bf16* qt, const bf16* kt, const b
                 const bf16* dot, const float* lse, const float* delta, const int32_t* sel,
                 const int32_t* key_offsets, const int32_t* query_lists, const float* dpooled,
                 bf16* dq, bf16* dk, bf16* dv, int* status, cudaStream_t s) {
-  static unsigned long long dq_set = 0, dkdv_set = 0;
+  static CtxCache<char> dq_set, dkdv_set;
   const int dq_bytes = dq_smem_floats<D>() * static_cast<int>(sizeof(float));
   const int dkdv_bytes = dkdv_smem_floats<D>() * static_cast<int>(sizeof(float));
   cudaError_t err = smem_limit_once(fine_bwd_dq<D>, dq_bytes, &dq_set);

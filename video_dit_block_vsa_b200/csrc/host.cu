@@ -9,14 +9,12 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <mutex>
 
 #include "common.cuh"
 
 namespace vsa {
 namespace {
 
-constexpr int kMaxDevices = 64;
 constexpr int kBufs = 2;  // chunk buffers in flight
 
 struct CopyStreams {
@@ -24,26 +22,21 @@ struct CopyStreams {
   cudaStream_t d2h = nullptr;
 };
 
-std::mutex g_streams_mu;
-CopyStreams g_streams[kMaxDevices];
+CtxCache<CopyStreams> g_streams;
 
-// Two non-blocking copy streams per device, created on first use and kept
-// for the life of the process.
+// Two non-blocking copy streams per CUDA context, created on first use in
+// that context and kept for the life of the process (a stream belongs to the
+// context it was created in).
 int copy_streams(CopyStreams* out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return VSA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_streams_mu);
-  CopyStreams& cs = g_streams[dev];
-  if (cs.h2d == nullptr) {
-    if (cudaStreamCreateWithFlags(&cs.h2d, cudaStreamNonBlocking) != cudaSuccess) return VSA_ERR_CUDA;
-    if (cudaStreamCreateWithFlags(&cs.d2h, cudaStreamNonBlocking) != cudaSuccess) {
-      cudaStreamDestroy(cs.h2d);
-      cs.h2d = nullptr;
-      return VSA_ERR_CUDA;
+  const bool ok = g_streams.get(current_context_id(), [](CopyStreams* cs) {
+    if (cudaStreamCreateWithFlags(&cs->h2d, cudaStreamNonBlocking) != cudaSuccess) return false;
+    if (cudaStreamCreateWithFlags(&cs->d2h, cudaStreamNonBlocking) != cudaSuccess) {
+      cudaStreamDestroy(cs->h2d);
+      return false;
     }
-  }
-  *out = cs;
-  return VSA_OK;
+    return true;
+  }, out);
+  return ok ? VSA_OK : VSA_ERR_CUDA;
 }
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }

@@ -11,11 +11,12 @@
 // the process exits.
 //
 // The array's host-side name is only a stand-in for the symbol, never a device
-// address, so the device address is looked up once per device with
-// cudaGetSymbolAddress (with that device current) and passed to the kernels.
-// The first call on each device does that lookup.
-#include <mutex>
-
+// address, so the device address is looked up with cudaGetSymbolAddress in the
+// calling thread's current CUDA context and passed to the kernels.  The
+// address belongs to that context, so it is cached per context (by the
+// context's unique id): a context the caller made current, or the new primary
+// context after cudaDeviceReset, gets its own lookup.  The first call in each
+// context does that lookup.
 #include "common.cuh"
 
 namespace vsa {
@@ -25,23 +26,14 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = 32ull << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDev = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDev];
+CtxCache<void*> g_noalloc_ptr;
 
-// Device address of the scratch array on the current device (set up once).
+// Device address of the scratch array in the current context.
 int noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return VSA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-      return VSA_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
-  return VSA_OK;
+  const bool ok = g_noalloc_ptr.get(current_context_id(), [](void** p) {
+    return cudaGetSymbolAddress(p, g_noalloc_scratch) == cudaSuccess && *p != nullptr;
+  }, out);
+  return ok ? VSA_OK : VSA_ERR_CUDA;
 }
 
 }  // namespace

@@ -176,7 +176,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
       : "memory");
 }
 
-// ---- generated: 16-lane TMEM access shapes (M = 64 accumulators)
+// ---- 16-lane TMEM access shapes (M = 64 accumulators)
 
 // TMEM -> registers, 16 lanes: threads 0-15 read lanes base..base+15 at
 // columns [col, col+32), threads 16-31 the same lanes at [col+32, col+64).

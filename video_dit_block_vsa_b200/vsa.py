@@ -494,6 +494,24 @@ def vsa_forward(shape, q, k, v, topk, out, g_fine=None, g_coarse=None, bufs=None
     return bufs
 
 
+def vsa_forward_fused(shape, q, k, v, topk, out, g_fine=None, g_coarse=None, bufs=None,
+                      stream=None):
+    """The whole path in the three launches the benchmark times: tiling with
+    the cube means in one pass, the coarse stage from those means, and the
+    fine kernel whose epilogue applies the gated combine and writes ``out``
+    in token order.  Same bits as ``vsa_forward``.  Returns the buffers."""
+    if bufs is None:
+        bufs = VsaBuffers(shape, topk, device=q.device, want_coarse=g_fine is not None)
+    vsa_tile_permute_pool(shape, q, k, v, bufs.q_t, bufs.k_t, bufs.v_t, bufs.workspace,
+                          bufs.counts, stream)
+    vsa_coarse_select_pooled(shape, topk, bufs.sel, bufs.workspace, o_coarse=bufs.o_c,
+                             stream=stream)
+    vsa_block_sparse_fwd_out(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, bufs.sel, topk,
+                             out, bufs.o_c if g_fine is not None else None, g_fine, g_coarse,
+                             stream=stream)
+    return bufs
+
+
 class VsaGradBuffers:
     """Device scratch of one backward call, allocated once with torch."""
 
