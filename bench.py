@@ -65,12 +65,20 @@ def cube_counts(grid):
     return (ct[:, None, None] * cy[None, :, None] * cx[None, None, :]).reshape(-1).astype(np.int64)
 
 
+def key_chunks(counts, sel):
+    """16-row key chunks the fine kernel loads and multiplies per query cube:
+    4 for a selected cube with more than 16 valid tokens, 1 otherwise."""
+    per_cube = np.where(counts > 16, 4, 1)
+    return per_cube[sel].sum(axis=-1)          # [B, H, C]
+
+
 def flop_counts(w, counts, sel):
-    """(fine effective FLOPs, fine issued FLOPs, coarse FLOPs) of one call."""
+    """(fine effective FLOPs, fine issued FLOPs, coarse FLOPs) of one call.
+    Issued: every query cube's 64 rows against its packed key chunks."""
     d, C = w.head_dim, counts.shape[0]
     nsel = counts[sel]                         # [B, H, C, k]
     fine_eff = 4.0 * d * float(np.sum(counts[None, None, :] * nsel.sum(axis=-1)))
-    fine_issued = 4.0 * d * w.batch * w.heads * C * w.topk * 64 * 64
+    fine_issued = 4.0 * d * 64 * 16 * float(key_chunks(counts, sel).sum())
     coarse = 4.0 * d * w.batch * w.heads * C * C
     return fine_eff, fine_issued, coarse
 
@@ -356,10 +364,11 @@ def run_gpu(args, w):
             traffic = tj.get("bytes_per_launch")
     except (OSError, ValueError):
         pass
-    # The fine kernel's other roofline: every selected K/V tile and every Q tile
-    # is moved from L2 into shared memory by TMA, and one SM's TMA path sustains
-    # TMA_INGEST_GBS_PER_SM with this kernel's box shape.
-    kv_bytes = float(w.batch * w.heads * w.cubes) * (w.topk * 2 + 1) * 64 * w.head_dim * 2
+    # The fine kernel's other roofline: every packed K/V chunk and every Q tile
+    # is moved from L2 into shared memory by TMA, and one SM sustains
+    # TMA_INGEST_GBS_PER_SM.
+    chunks = float(key_chunks(counts, bufs.sel.cpu().numpy().astype(np.int64)).sum())
+    kv_bytes = (chunks * 2 * 16 + float(w.batch * w.heads * w.cubes) * 64) * w.head_dim * 2
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     feed_peak = TMA_INGEST_GBS_PER_SM * sms / 1e3
     feed = {"path": "L2 -> shared memory (TMA)", "bytes": kv_bytes,
@@ -423,9 +432,9 @@ def run_gpu(args, w):
     return 0
 
 
-# Sustained TMA ingest of one SM for random 64-row x 128-byte swizzled boxes from
-# L2, measured on B200 (the best of two probe layouts; the figure did not move
-# with 2 to 6 ring slots or with 37 to 148 SMs loading at once).
+# Sustained TMA ingest of one SM for random 64-row x 128-byte swizzled boxes
+# from L2, measured on B200 with one issuing thread filling a ring of 32 KB
+# slots (148 SMs loading at once): the best of the probe layouts, 99.3 GB/s.
 TMA_INGEST_GBS_PER_SM = 99.3
 
 # (b, h) planes per chunk of the host-buffer path in the end-to-end leg.
@@ -515,7 +524,7 @@ def run_backward_pieces(args, w):
 
 # Revision tag of the fine kernel; ncu traffic figures are only reported for
 # the revision they were captured on.
-KERNEL_REV = "fine-v3.2-out"
+KERNEL_REV = "fine-v5-packed-out"
 
 
 def main():

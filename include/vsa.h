@@ -100,8 +100,12 @@ int vsa_tile_permute(const vsa_shape* shape, const void* x, void* x_tiled,
  * tokens (qbar, kbar, vbar); coarse attention over the C pooled vectors with
  * scale 1/sqrt(d) gives the coarse output O_c = softmax(qbar kbar^T/sqrt(d)) vbar;
  * for each query cube the k key cubes with the largest coarse logits are
- * selected, ties to the lower index, listed in ascending index order.
- * Logits are computed in float32.
+ * selected, ties to the lower index.  Each row lists the selected key cubes
+ * that hold more than 16 valid tokens first, then the others, each group in
+ * ascending index order (the order in which the fine stage packs key rows:
+ * a cube of at most 16 tokens costs it a quarter of a full cube; on a grid
+ * whose sides are multiples of 4 every cube is full and the order is plain
+ * ascending).  Logits are computed in float32.
  *   q_tiled, k_tiled, v_tiled  bf16 [B, H, 64*C, d] from vsa_tile_permute
  *   cube_count   int32 [C] as written by vsa_tile_permute for this shape
  *                (checked against the grid; a mismatch is recorded as
@@ -187,9 +191,15 @@ int vsa_coarse_select_noalloc(const vsa_shape* shape, const void* q_tiled, const
  * rows are written as 0.  bf16 in, float32 accumulation, bf16 out.
  *   q_tiled, k_tiled, v_tiled  bf16 [B, H, 64*C, d]
  *   cube_count   int32 [C] (checked as in vsa_coarse_select)
- *   sel_idx      int32 [B, H, C, k], each row strictly ascending in [0, C)
- *                (an entry out of range or out of order is recorded as
- *                VSA_ERR_BAD_INDEX; out-of-range entries are clamped)
+ *   sel_idx      int32 [B, H, C, k], entries in [0, C), each row in the
+ *                order vsa_coarse_select writes: key cubes with more than 16
+ *                valid tokens first, then the others, each group strictly
+ *                ascending (an entry out of range or out of order is recorded
+ *                as VSA_ERR_BAD_INDEX; out-of-range entries are clamped)
+ * The kernel packs the key rows of a query cube's selection into 128-row
+ * steps: a cube of more than 16 tokens takes 64 rows, one of at most 16 takes
+ * 16 rows, so the partial cubes at the edges of a ragged grid cost a quarter
+ * of a full cube.
  *   o_fine_tiled bf16 [B, H, 64*C, d] (written)
  *   lse          float32 [B, H, 64*C] natural-log log-sum-exp of each valid
  *                row's scaled scores (-inf for pad rows), or NULL */
@@ -265,9 +275,9 @@ int vsa_forward_host(const vsa_shape* shape, int topk, const void* q, const void
  * for every key cube j of every (b, h), the query cubes i with j in
  * sel_idx[b, h, i, :], in ascending order, as a CSR list.  The pages have no
  * counterpart (they describe no backward kernel); it is a building block.
- *   sel_idx      int32 [B, H, C, k], rows ascending without repeats (as
- *                vsa_coarse_select writes them); an index outside [0, C) is
- *                recorded as VSA_ERR_BAD_INDEX and left out
+ *   sel_idx      int32 [B, H, C, k], rows without repeats, in any order (for
+ *                example as vsa_coarse_select writes them); an index outside
+ *                [0, C) is recorded as VSA_ERR_BAD_INDEX and left out
  *   key_offsets  int32 [B, H, C + 1] (written): key cube j's list is
  *                query_lists[b, h, key_offsets[b, h, j] .. key_offsets[b, h, j + 1])
  *   query_lists  int32 [B, H, C * k] (written)

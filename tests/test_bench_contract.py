@@ -32,7 +32,7 @@ def test_reference_arm_prints_one_contract_line():
 
 def test_flop_accounting_counts_valid_token_pairs():
     # effective FLOPs = 4 d x (number of (query token, selected key token) pairs
-    # over valid tokens); issued FLOPs count every 64x64 tile in full
+    # over valid tokens)
     import numpy as np
     sys.path.insert(0, ROOT)
     import bench
@@ -53,5 +53,12 @@ def test_flop_accounting_counts_valid_token_pairs():
                 for j in sel[b, h, i]:
                     pairs += int(counts[i]) * int(counts[j])
     assert eff == 4.0 * w.head_dim * pairs
-    assert issued == 4.0 * w.head_dim * 2 * 3 * C * w.topk * 64 * 64
+    # issued: 64 query rows x the packed key rows (a selected cube with more
+    # than 16 valid tokens costs 64 key rows, one with at most 16 costs 16)
+    rows = 0
+    for b in range(2):
+        for h in range(3):
+            for i in range(C):
+                rows += sum(64 if counts[j] > 16 else 16 for j in sel[b, h, i])
+    assert issued == 4.0 * w.head_dim * 64 * rows
     assert coarse == 4.0 * w.head_dim * 2 * 3 * C * C

@@ -11,7 +11,7 @@ import torch
 
 from oracle import vsa_oracle as vo
 from video_dit_block_vsa_b200 import workloads as wl
-from tests.vsa_checks import (assert_close, bf16_dev_bits, bf16_dev_to_f64, check_selection,
+from tests.vsa_checks import (assert_close, bf16_dev_bits, bf16_dev_to_f64, check_selection, wide_first,
                               to_dev_bf16)
 
 pytestmark = pytest.mark.gpu
@@ -111,7 +111,7 @@ def test_coarse_select(vsa, B, H, d, grid, k):
     assert_close(ws[1], kb, "kbar", 1e-5, 1e-6)
     assert_close(ws[2], vb, "vbar", 1e-5, 1e-6)
     assert_close(logits.cpu().numpy(), S, "coarse logits", 2e-5, 2e-6)
-    equal, swapped = check_selection(bufs.sel.cpu().numpy(), S, k)
+    equal, swapped = check_selection(bufs.sel.cpu().numpy(), S, k, counts)
     assert equal + swapped == B * H * C
     assert_close(bufs.o_c.cpu().numpy(), O_c, "coarse output", 1e-4, 1e-5)
     assert vsa.vsa_get_status() == 0
@@ -204,7 +204,8 @@ def test_topk_ties_go_to_lower_index(vsa, grid, k):
     vsa.vsa_tile_permute(shape, to_dev_bf16(kv), bufs.v_t)
     vsa.vsa_coarse_select(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, k, bufs.sel, bufs.workspace)
     sel = bufs.sel.cpu().numpy()
-    assert np.all(sel == np.arange(k))
+    # the k lowest indices, listed wide cubes first (each group ascending)
+    assert np.all(sel == wide_first(np.arange(k), vo.cube_permutation(grid)[1]))
 
 
 # --------------------------------------------------------------------------
@@ -220,6 +221,8 @@ def fine_case(vsa, B, H, d, grid, sel_np, seed=9, lse=True):
     bufs = vsa.VsaBuffers(shape, k, want_lse=lse)
     for n, t in (("q", bufs.q_t), ("k", bufs.k_t), ("v", bufs.v_t)):
         vsa.vsa_tile_permute(shape, to_dev_bf16(x[n]), t, bufs.counts if n == "q" else None)
+    _, grid_counts = vo.cube_permutation(grid)
+    sel_np = wide_first(sel_np, grid_counts)  # the fine kernel's row order
     bufs.sel.copy_(torch.from_numpy(sel_np.astype(np.int32)))
     bufs.o_f.fill_(float("nan"))
     vsa.vsa_block_sparse_fwd(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, bufs.sel, k,
@@ -386,7 +389,7 @@ def check_workload(vsa, w, head_sample=None, cube_sample=None):
         q_t, k_t, v_t = tiled["q"], tiled["k"], tiled["v"]
         S, O_c = vo.coarse_attention(vo.pool(q_t, counts), vo.pool(k_t, counts), vo.pool(v_t, counts))
         sel = sel_gpu[b:b + 1, h:h + 1]
-        check_selection(sel, S, w.topk)  # selection up to ties; outputs use the GPU's choice
+        check_selection(sel, S, w.topk, counts)  # selection up to ties; outputs use the GPU's choice
         if (b, h) not in sampled:
             continue
         gf = x["g_f"][b:b + 1, h:h + 1].astype(np.float64) if w.gated else None

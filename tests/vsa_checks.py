@@ -28,19 +28,34 @@ def bf16_dev_bits(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-def check_selection(sel_gpu: np.ndarray, logits_ref: np.ndarray, k: int):
+def wide_first(sel: np.ndarray, counts: np.ndarray) -> np.ndarray:
+    """The library's order of a selection row: key cubes with more than 16
+    valid tokens first, then the others, each group ascending (the order the
+    fine kernel packs key rows in).  Same set, rows reordered."""
+    sel = np.asarray(sel)
+    narrow = (np.asarray(counts)[sel] <= 16).astype(np.int64)
+    order = np.lexsort((sel, narrow), axis=-1)
+    return np.take_along_axis(sel, order, axis=-1)
+
+
+def check_selection(sel_gpu: np.ndarray, logits_ref: np.ndarray, k: int, counts=None):
     """Accepts the GPU's per-row selection if it is a top-k set of the
-    reference logits up to the tie band.  Returns (rows_equal, rows_tie_swapped).
+    reference logits up to the tie band, listed in the library's order (wide
+    key cubes first, each group ascending; with counts None every cube counts
+    as wide, i.e. plain ascending).  Returns (rows_equal, rows_tie_swapped).
     Raises AssertionError with the first offending row otherwise."""
     C = logits_ref.shape[-1]
+    if counts is None:
+        counts = np.full(C, 64)
     flat_sel = sel_gpu.reshape(-1, k)
     flat_s = logits_ref.reshape(-1, C)
     equal = swapped = 0
-    ref_sel = vo.topk_select(flat_s, k)
+    ref_sel = wide_first(vo.topk_select(flat_s, k), counts)
     for r in range(flat_sel.shape[0]):
         g = flat_sel[r]
-        assert np.all(np.diff(g) > 0), f"row {r}: selection not strictly ascending: {g}"
         assert g.min() >= 0 and g.max() < C, f"row {r}: index out of range"
+        assert np.array_equal(g, wide_first(g, counts)), f"row {r}: not in wide-first ascending order: {g}"
+        assert np.unique(g).size == k, f"row {r}: repeated index: {g}"
         if np.array_equal(g, ref_sel[r]):
             equal += 1
             continue

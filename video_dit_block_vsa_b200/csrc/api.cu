@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "fine.cuh"
 
 namespace vsa {
 
@@ -23,10 +24,9 @@ cudaError_t launch_tile_pool(const Geom&, const void*, const void*, const void*,
                              void*, int32_t*, float*, int*, cudaStream_t);
 cudaError_t launch_coarse_only(const Geom&, int, float*, int32_t*, float*, const float*,
                                cudaStream_t);
-cudaError_t launch_block_sparse_fwd(const Geom&, const CUtensorMap&, const CUtensorMap&,
-                                    const CUtensorMap&, const int32_t*, const int32_t*, int,
-                                    void*, float*, const float*, const float*, const float*, bool,
-                                    int*, int, cudaStream_t);
+cudaError_t launch_block_sparse_fwd(const Geom&, const FineMaps&, const int32_t*, const int32_t*,
+                                    int, void*, float*, const float*, const float*, const float*,
+                                    bool, int*, int, cudaStream_t);
 cudaError_t launch_debug_wait(uint64_t, int*, cudaStream_t);
 cudaError_t launch_select_transpose(int, int, int, const int32_t*, int32_t*, int32_t*, int32_t*,
                                     int*, cudaStream_t);
@@ -157,17 +157,26 @@ int make_geom(const vsa_shape* s, Geom* g) {
   return VSA_OK;
 }
 
-int tiled_map(const Geom& g, const void* ptr, CUtensorMap* m) {
+int tiled_map(const Geom& g, const void* ptr, CUtensorMap* m, int box_rows = 64) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(g.d),
                               static_cast<cuuint64_t>(g.B) * g.H * g.rows};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(g.d) * 2};
-  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
                               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;
+}
+
+// The fine kernel's maps: q, k, v with one-cube boxes, k and v with 16-row boxes.
+int fine_maps(const Geom& g, const void* q, const void* k, const void* v, FineMaps* m) {
+  if (tiled_map(g, q, &m->q) != VSA_OK || tiled_map(g, k, &m->k) != VSA_OK ||
+      tiled_map(g, v, &m->v) != VSA_OK || tiled_map(g, k, &m->k16, 16) != VSA_OK ||
+      tiled_map(g, v, &m->v16, 16) != VSA_OK)
+    return VSA_ERR_CUDA;
+  return VSA_OK;
 }
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA; }
@@ -369,11 +378,9 @@ int vsa_block_sparse_fwd(const vsa_shape* shape, const void* q_tiled, const void
   DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   if ((rc = get_encoder()) != VSA_OK) return rc;
-  CUtensorMap tq, tk, tv;
-  if (tiled_map(g, q_tiled, &tq) != VSA_OK || tiled_map(g, k_tiled, &tk) != VSA_OK ||
-      tiled_map(g, v_tiled, &tv) != VSA_OK)
-    return VSA_ERR_CUDA;
-  return cuda_rc(launch_block_sparse_fwd(g, tq, tk, tv, cube_count, sel_idx, topk, o_fine_tiled,
+  FineMaps maps;
+  if (fine_maps(g, q_tiled, k_tiled, v_tiled, &maps) != VSA_OK) return VSA_ERR_CUDA;
+  return cuda_rc(launch_block_sparse_fwd(g, maps, cube_count, sel_idx, topk, o_fine_tiled,
                                          lse, nullptr, nullptr, nullptr, false, st.status, st.sms,
                                          stream));
 }
@@ -401,11 +408,9 @@ int vsa_block_sparse_fwd_out(const vsa_shape* shape, const void* q_tiled, const 
   DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   if ((rc = get_encoder()) != VSA_OK) return rc;
-  CUtensorMap tq, tk, tv;
-  if (tiled_map(g, q_tiled, &tq) != VSA_OK || tiled_map(g, k_tiled, &tk) != VSA_OK ||
-      tiled_map(g, v_tiled, &tv) != VSA_OK)
-    return VSA_ERR_CUDA;
-  return cuda_rc(launch_block_sparse_fwd(g, tq, tk, tv, cube_count, sel_idx, topk, out, lse,
+  FineMaps maps;
+  if (fine_maps(g, q_tiled, k_tiled, v_tiled, &maps) != VSA_OK) return VSA_ERR_CUDA;
+  return cuda_rc(launch_block_sparse_fwd(g, maps, cube_count, sel_idx, topk, out, lse,
                                          g_fine ? o_coarse : nullptr, g_fine, g_coarse, true,
                                          st.status, st.sms, stream));
 }

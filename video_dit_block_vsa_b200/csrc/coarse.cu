@@ -105,11 +105,13 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 constexpr int kTopkRegs = 48;
 
 // Writes the indices of the k largest of row[0..C) (ties: lower index first)
-// in ascending order to out[0..k).  Executed by one full warp; hist is a
-// warp-private 256-entry smem array.  Most-significant-digit-first radix
+// to out[0..k): first the key cubes holding more than 16 valid tokens, then
+// the others, each group in ascending order.  Executed by one full warp; hist
+// is a warp-private 256-entry smem array.  Most-significant-digit-first radix
 // select over the order-preserving integer image of the floats, 8 bits per
-// pass, then one ballot-compaction pass in index order.
-__device__ void warp_topk(const float* row, int C, int k, int* hist, int32_t* out) {
+// pass, then two ballot-compaction passes in index order.
+__device__ void warp_topk(const Geom& g, const float* row, int C, int k, int* hist,
+                          int32_t* out) {
   const int lane = threadIdx.x & 31;
   uint32_t kc[kTopkRegs];
 #pragma unroll
@@ -169,33 +171,42 @@ __device__ void warp_topk(const float* row, int C, int k, int* hist, int32_t* ou
     __syncwarp();
   }
   // prefix = key of the k-th largest; take all keys above it and the first
-  // `remaining` keys equal to it, in index order.
+  // `remaining` keys equal to it in index order.  The taken keys are written
+  // in two passes, the key cubes with more than 16 valid tokens first, then
+  // the others, each in ascending index order (the order the fine kernel
+  // packs key rows in); which keys are taken does not depend on the pass.
   const unsigned lt = (1u << lane) - 1u;
-  int pos = 0, eq_seen = 0;
+  auto emit = [&](bool want_wide, int pos) -> int {
+    int eq_seen = 0;
 #pragma unroll
-  for (int u = 0; u < kTopkRegs; ++u) {
-    const int j = lane + 32 * u;
-    const bool gt = j < C && kc[u] > prefix;
-    const bool eq = j < C && kc[u] == prefix;
-    const unsigned eqm = __ballot_sync(0xffffffffu, eq);
-    const bool take = gt || (eq && eq_seen + __popc(eqm & lt) < remaining);
-    const unsigned tm = __ballot_sync(0xffffffffu, take);
-    if (take) out[pos + __popc(tm & lt)] = j;
-    pos += __popc(tm);
-    eq_seen += __popc(eqm);
-  }
-  for (int j0 = 32 * kTopkRegs; j0 < C; j0 += 32) {
-    const int j = j0 + lane;
-    const uint32_t key = j < C ? order_key(row[j]) : 0u;
-    const bool gt = j < C && key > prefix;
-    const bool eq = j < C && key == prefix;
-    const unsigned eqm = __ballot_sync(0xffffffffu, eq);
-    const bool take = gt || (eq && eq_seen + __popc(eqm & lt) < remaining);
-    const unsigned tm = __ballot_sync(0xffffffffu, take);
-    if (take) out[pos + __popc(tm & lt)] = j;
-    pos += __popc(tm);
-    eq_seen += __popc(eqm);
-  }
+    for (int u = 0; u < kTopkRegs; ++u) {
+      const int j = lane + 32 * u;
+      const bool gt = j < C && kc[u] > prefix;
+      const bool eq = j < C && kc[u] == prefix;
+      const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+      const bool take = (gt || (eq && eq_seen + __popc(eqm & lt) < remaining)) &&
+                        ((cube_valid(g, j < C ? j : 0) > 16) == want_wide);
+      const unsigned tm = __ballot_sync(0xffffffffu, take);
+      if (take) out[pos + __popc(tm & lt)] = j;
+      pos += __popc(tm);
+      eq_seen += __popc(eqm);
+    }
+    for (int j0 = 32 * kTopkRegs; j0 < C; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t key = j < C ? order_key(row[j]) : 0u;
+      const bool gt = j < C && key > prefix;
+      const bool eq = j < C && key == prefix;
+      const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+      const bool take = (gt || (eq && eq_seen + __popc(eqm & lt) < remaining)) &&
+                        ((cube_valid(g, j < C ? j : 0) > 16) == want_wide);
+      const unsigned tm = __ballot_sync(0xffffffffu, take);
+      if (take) out[pos + __popc(tm & lt)] = j;
+      pos += __popc(tm);
+      eq_seen += __popc(eqm);
+    }
+    return pos;
+  };
+  emit(false, emit(true, 0));
 }
 
 // ------------------------------------------------------------------ coarse
@@ -299,7 +310,7 @@ __global__ void __launch_bounds__(kCoarseThreads) coarse_kernel(
   // ---- top-k on the logits, then softmax in place (one warp per row)
   for (int r = warp; r < rows; r += 8) {
     float* row = S + static_cast<size_t>(r) * Cp;
-    warp_topk(row, C, topk, hist + warp * 256,
+    warp_topk(g, row, C, topk, hist + warp * 256,
               sel + (static_cast<long long>(bh) * C + i0 + r) * topk);
     float mx = -INFINITY;
 #pragma unroll 8

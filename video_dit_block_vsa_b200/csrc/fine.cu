@@ -10,10 +10,19 @@
 //    so that the tensor core works on one while the other's softmax runs.
 //  * Warp roles: warp 0 = TMA producer, warp 1 = MMA issuer (one thread),
 //    warps 4-7 = softmax of cube A, warps 8-11 = softmax of cube B.
-//  * A "step" covers two selected key cubes (128 keys, one N = 128 MMA;
-//    an odd k ends with a 64-key step).  Keys and values stream through a
-//    ring of 128-key smem slots (128-byte swizzle, TMA-filled) in exactly the
-//    order the MMA issuer consumes them: K_A0 K_B0 | V_A0 K_A1 V_B0 K_B1 | ...
+//  * Key packing: each selected key cube is "wide" (more than 16 valid tokens:
+//    one 64-row group of four 16-row chunks) or "narrow" (at most 16 valid
+//    tokens, packed to the front of the cube: one 16-row chunk).  A selection
+//    row lists its wide cubes first (the coarse stage writes them that way), so
+//    a cube's key rows are a sequence of T = 4 W + (k - W) chunks and step j
+//    holds chunks 8j .. 8j+7: 128 key rows, one N = 128 MMA.  The partial
+//    cubes of a ragged grid so cost a quarter of a full cube.  The last step
+//    of a cube may hold fewer chunks: its Q K^T uses N = 16 x chunks and its
+//    P V that many 16-key slices.  The two cubes of an item may have
+//    different step counts.
+//  * Keys and values stream through a ring of 128-key smem slots (128-byte
+//    swizzle, TMA-filled) in exactly the order the MMA issuer consumes them:
+//    K_A0 K_B0 | V_A0 K_A1 V_B0 K_B1 | ...
 //  * TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+d),
 //    O_B [256+d, 256+2d).  The softmax writes P (bf16 pairs) over the first 64
 //    columns of its S, and O += P V reads P straight from TMEM (A operand in
@@ -32,6 +41,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "fine.cuh"
 #include "ptx.cuh"
 
 namespace vsa {
@@ -49,6 +59,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleLog2 = 8.0f;  // rescale only when a row max grows by > 2^8
+constexpr int kWideMin = 17;          // a key cube with this many valid tokens or more is wide
 
 template <int D>
 struct Cfg {
@@ -60,7 +71,7 @@ struct Cfg {
   static constexpr int kSlots = D == 128 ? 5 : 10;
   static constexpr uint32_t kRingOff = 4 * kQBytes;            // Q: 2 items x 2 cubes
   static constexpr uint32_t kBarOff = kRingOff + kSlots * kSlotBytes;
-  static constexpr size_t kSmem = 1024 + kBarOff + 320;
+  static constexpr size_t kSmem = 1024 + kBarOff + 336;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128;
   static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(64, D, false, true);  // P (TMEM), V MN-major
@@ -79,6 +90,7 @@ struct OutSpec {
 };
 
 struct Shared {
+  volatile int* chunks;  // [2 Q buffers][2 cubes]: 16-row key chunks, producer -> MMA thread
   uint64_t* q_full;
   uint64_t* q_empty;
   uint64_t* kv_full;
@@ -124,41 +136,105 @@ __device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&p);
 }
 
-// ------------------------------------------------------------------ producer
-// Selection indices of one list, fetched 32 at a time into the lanes of the
-// producer warp (one index per lane) with the next window already in flight,
-// so the slot loads never wait on a global load.
-struct IndexWindow {
-  const int32_t* list;
-  int base, cur, nxt;
+__device__ __forceinline__ int clamp_cube(const Geom& g, int x) {
+  return x < 0 ? 0 : (x >= g.C ? g.C - 1 : x);
+}
+
+// ------------------------------------------------------------------ key plan
+// A selection row lists its W wide key cubes first, then its k - W narrow
+// ones (each group ascending, as the coarse stage writes it).  The cube's key
+// rows are a sequence of T = 4 W + (k - W) chunks of 16 rows; step j holds
+// chunks 8j .. 8j+7, half h of it the four chunks from cb = 8j + 4h, which are
+// either one wide cube (cb < 4W) or up to four narrow ones.
+
+// What half-step from chunk cb holds: 0 nothing, 1 one wide cube, 2 narrow cubes.
+__device__ __forceinline__ int half_kind(int cb, int W, int T) {
+  return cb >= T ? 0 : (cb < 4 * W ? 1 : 2);
+}
+
+// List entry of chunk slot q (0..3) of the half-step from chunk cb, or -1
+// (the three continuation slots of a wide cube and slots past the end).
+__device__ __forceinline__ int half_entry(int cb, int q, int W, int topk) {
+  if (cb < 4 * W) return q == 0 ? cb >> 2 : -1;
+  const int e = W + (cb - 4 * W) + q;
+  return e < topk ? e : -1;
+}
+
+// Key cube of list entry e (clamped into [0, C); the producer reports bad
+// entries), or -1 for e < 0.
+__device__ __forceinline__ int entry_cube(const Geom& g, const int32_t* list, int e) {
+  return e < 0 ? -1 : clamp_cube(g, __ldg(&list[e]));
+}
+
+// Wide entries of a list (warp-collective).  With `status`, also checks the
+// list: entries in [0, C), wide cubes before narrow ones, each group strictly
+// ascending; a violation is recorded as VSA_ERR_BAD_INDEX.  The loads of up
+// to eight 32-entry windows are issued before any of them is used.
+__device__ __forceinline__ int count_wide(const Geom& g, const int32_t* list, int topk, int lane,
+                                          int* status) {
+  int wide = 0;
+  int prev_last = -1;
+  bool prev_wide_last = true;
+  bool bad = false;
+  for (int b0 = 0; b0 < topk; b0 += 256) {
+    int raws[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = b0 + 32 * u + lane;
+      raws[u] = i < topk ? __ldg(&list[i]) : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int b = b0 + 32 * u;
+      if (b >= topk) break;
+      const bool in = b + lane < topk;
+      const int raw = raws[u];
+      const bool w = in && cube_valid(g, clamp_cube(g, raw)) >= kWideMin;
+      wide += __popc(__ballot_sync(0xffffffffu, w));
+      if (status != nullptr) {
+        int prev = __shfl_up_sync(0xffffffffu, raw, 1);
+        bool prev_w = __shfl_up_sync(0xffffffffu, w, 1);
+        if (lane == 0) {
+          prev = prev_last;
+          prev_w = prev_wide_last;
+        }
+        if (in) {
+          bad |= raw < 0 || raw >= g.C;
+          if (b + lane > 0) bad |= (w && !prev_w) || (w == prev_w && raw <= prev);
+        }
+        prev_last = __shfl_sync(0xffffffffu, raw, 31);
+        prev_wide_last = __shfl_sync(0xffffffffu, w, 31);
+      }
+    }
+  }
+  if (status != nullptr && __any_sync(0xffffffffu, bad) && lane == 0)
+    report(status, VSA_ERR_BAD_INDEX);
+  return wide;
+}
+
+// A list entry fetched ahead of its use: the load is issued now and the value
+// (clamped into [0, C)) is only read by `cube_of` later, so the load's latency
+// overlaps other work.
+struct Ahead {
+  int raw;
+  bool present;
 };
 
-__device__ __forceinline__ int fetch_index(const int32_t* list, int i, int topk) {
-  return i < topk ? __ldg(&list[i]) : 0;
+__device__ __forceinline__ Ahead fetch_entry(const int32_t* list, int e) {
+  Ahead a;
+  a.present = e >= 0;
+  a.raw = a.present ? __ldg(&list[e]) : 0;
+  return a;
 }
 
-__device__ __forceinline__ void window_init(IndexWindow& w, const int32_t* list, int topk,
-                                            int lane) {
-  w.list = list;
-  w.base = 0;
-  w.cur = fetch_index(list, lane, topk);
-  w.nxt = fetch_index(list, 32 + lane, topk);
+__device__ __forceinline__ int cube_of(const Geom& g, const Ahead& a) {
+  return a.present ? clamp_cube(g, a.raw) : -1;
 }
 
-// Warp-collective: returns list[a] on every lane; a never decreases.
-__device__ __forceinline__ int window_get(IndexWindow& w, int a, int topk, int lane) {
-  while (a >= w.base + 32) {
-    w.base += 32;
-    w.cur = w.nxt;
-    w.nxt = fetch_index(w.list, w.base + 32 + lane, topk);
-  }
-  return __shfl_sync(0xffffffffu, w.cur, a - w.base);
-}
-
+// ------------------------------------------------------------------ producer
 // Run by the whole producer warp; lane 0 issues the barrier and TMA operations.
 template <int D>
-__device__ void producer(const Shared& sh, const Geom& g, const CUtensorMap* tq,
-                         const CUtensorMap* tk, const CUtensorMap* tv,
+__device__ void producer(const Shared& sh, const Geom& g, const FineMaps& maps,
                          const int32_t* __restrict__ counts, const int32_t* __restrict__ sel,
                          int topk, int* status) {
   using Cf = Cfg<D>;
@@ -166,7 +242,6 @@ __device__ void producer(const Shared& sh, const Geom& g, const CUtensorMap* tq,
   const bool leader = lane == 0;
   const int pairs = (g.C + 1) / 2;
   const int items = g.B * g.H * pairs;
-  const int nsteps = (topk + 1) / 2;
   uint32_t ring = 0;
   int t = 0;
   // lane 0 waits; the verdict is broadcast so the warp leaves together
@@ -181,63 +256,98 @@ __device__ void producer(const Shared& sh, const Geom& g, const CUtensorMap* tq,
     if (leader && (__ldg(&counts[it.i0]) != cube_valid(g, it.i0) ||
                    (it.has_b && __ldg(&counts[it.i1]) != cube_valid(g, it.i1))))
       report(status, VSA_ERR_BAD_INDEX);
-    IndexWindow win[2];
-    const int32_t* list0 = sel + (static_cast<long long>(it.bh) * g.C + it.i0) * topk;
-    window_init(win[0], list0, topk, lane);
-    window_init(win[1], it.has_b ? list0 + topk : list0, topk, lane);
+    const int32_t* list[2];
+    list[0] = sel + (static_cast<long long>(it.bh) * g.C + it.i0) * topk;
+    list[1] = list[0] + topk;
+    int W[2], T[2], n[2];
+    W[0] = count_wide(g, list[0], topk, lane, status);
+    W[1] = it.has_b ? count_wide(g, list[1], topk, lane, status) : 0;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      T[c] = 3 * W[c] + topk;
+      n[c] = (T[c] + 7) / 8;
+    }
+    if (!it.has_b) T[1] = n[1] = 0;  // no cube B: nothing to plan or fetch
     // ---- query tiles of both cubes
     const int qb = t & 1;
     if (!wait_all(&sh.q_empty[qb], ((t >> 1) & 1) ^ 1)) return fail(sh, status);
     if (leader) {
+      sh.chunks[2 * qb] = T[0];  // published to the MMA thread by the q_full arrive
+      sh.chunks[2 * qb + 1] = it.has_b ? T[1] : 0;
       mbar_arrive_expect_tx(&sh.q_full[qb], (it.has_b ? 2 : 1) * Cf::kQBytes);
       uint8_t* qdst = sh.base + qb * 2 * Cf::kQBytes;
 #pragma unroll
       for (int h = 0; h < Cf::kHalves; ++h) {
-        tma_load_2d(qdst + h * Cf::kQHalf, tq, &sh.q_full[qb], h * 64, it.row0 + it.i0 * 64);
+        tma_load_2d(qdst + h * Cf::kQHalf, &maps.q, &sh.q_full[qb], h * 64, it.row0 + it.i0 * 64);
         if (it.has_b)
-          tma_load_2d(qdst + Cf::kQBytes + h * Cf::kQHalf, tq, &sh.q_full[qb], h * 64,
+          tma_load_2d(qdst + Cf::kQBytes + h * Cf::kQHalf, &maps.q, &sh.q_full[qb], h * 64,
                       it.row0 + it.i1 * 64);
       }
     }
-    // ---- key / value slots, in the MMA issuer's order
-    int prev[2] = {-1, -1};
-    auto load = [&](int c, int j, bool is_v) -> bool {
+    // ---- key / value slots, in the MMA issuer's order: K_A0 K_B0, then per
+    // step j: V_Aj K_A(j+1) V_Bj K_B(j+1), skipping steps a cube does not have.
+    // Lane q < 8 owns chunk slot q: its list entry for the next K load of each
+    // cube is fetched one K load ahead, and a V load reuses the entries of the
+    // K load of the same step.
+    auto lookup = [&](int c, int j) -> Ahead {
+      const int Wc = c ? W[1] : W[0], Tc = c ? T[1] : T[0];
+      const int cb = 8 * j + 4 * (lane >> 2);
+      int e = -1;
+      if (lane < 8 && half_kind(cb, Wc, Tc) != 0) e = half_entry(cb, lane & 3, Wc, topk);
+      return fetch_entry(c ? list[1] : list[0], e);
+    };
+    Ahead next_k[2] = {lookup(0, 0), lookup(1, 0)};
+    Ahead last_k[2] = {next_k[0], next_k[1]};
+    const int nmax = max(n[0], n[1]);
+    for (int e = 0;; ++e) {
+      int c, j;
+      bool is_v;
+      if (e < 2) {
+        c = e;
+        j = 0;
+        is_v = false;
+      } else {
+        const int js = (e - 2) >> 2, r = (e - 2) & 3;
+        if (js >= nmax) break;
+        c = r >> 1;
+        is_v = (r & 1) == 0;
+        j = is_v ? js : js + 1;
+      }
+      if (j >= (c ? n[1] : n[0])) continue;
+      if (*sh.abort_flag) return;
       const int slot = static_cast<int>(ring % Cf::kSlots);
       const uint32_t round = ring / Cf::kSlots;
       ++ring;
-      const int a = 2 * j;
-      const int nk = (a + 1 < topk) ? 2 : 1;
-      int jr[2];
-      jr[0] = window_get(win[c], a, topk, lane);
-      jr[1] = window_get(win[c], a + nk - 1, topk, lane);
-      if (!wait_all(&sh.kv_empty[slot], (round & 1u) ^ 1u)) return false;
-      if (leader) {
-        mbar_arrive_expect_tx(&sh.kv_full[slot], nk * 64 * D * 2);
-        uint8_t* dst = sh.base + Cf::kRingOff + slot * Cf::kSlotBytes;
-        for (int r = 0; r < nk; ++r) {
-          int x = jr[r];
-          if (!is_v) {  // validate once per index (on the key load)
-            if (x < 0 || x >= g.C || x <= prev[c]) report(status, VSA_ERR_BAD_INDEX);
-            prev[c] = x;
-          }
-          x = x < 0 ? 0 : (x >= g.C ? g.C - 1 : x);
-#pragma unroll
-          for (int h = 0; h < Cf::kHalves; ++h)
-            tma_load_2d(dst + h * Cf::kKVHalf + r * (64 * 128), is_v ? tv : tk,
-                        &sh.kv_full[slot], h * 64, it.row0 + x * 64);
+      // this step's chunk slots: lane q < 8 loads slot q's key cube
+      const int Wc = c ? W[1] : W[0], Tc = c ? T[1] : T[0];
+      const int cb0 = 8 * j;
+      const bool wide = half_kind(cb0 + 4 * (lane >> 2), Wc, Tc) == 1;
+      int mine;
+      if (is_v) {
+        mine = cube_of(g, c ? last_k[1] : last_k[0]);
+      } else {
+        const Ahead cur = c ? next_k[1] : next_k[0];
+        mine = cube_of(g, cur);
+        if (c) {
+          last_k[1] = cur;
+          next_k[1] = lookup(1, j + 1);
+        } else {
+          last_k[0] = cur;
+          next_k[0] = lookup(0, j + 1);
         }
       }
-      return true;
-    };
-    if (!load(0, 0, false)) return fail(sh, status);
-    if (it.has_b && !load(1, 0, false)) return fail(sh, status);
-    for (int j = 0; j < nsteps; ++j) {
-      if (*sh.abort_flag) return;
-      if (!load(0, j, true)) return fail(sh, status);
-      if (j + 1 < nsteps && !load(0, j + 1, false)) return fail(sh, status);
-      if (it.has_b) {
-        if (!load(1, j, true)) return fail(sh, status);
-        if (j + 1 < nsteps && !load(1, j + 1, false)) return fail(sh, status);
+      const int nc = min(8, Tc - cb0);
+      if (!wait_all(&sh.kv_empty[slot], (round & 1u) ^ 1u)) return fail(sh, status);
+      // the step's key rows: 64 per wide cube, 16 per narrow cube
+      if (leader) mbar_arrive_expect_tx(&sh.kv_full[slot], static_cast<uint32_t>(nc) * 16u * D * 2u);
+      __syncwarp();
+      if (mine >= 0) {
+        uint8_t* dst = sh.base + Cf::kRingOff + slot * Cf::kSlotBytes + (lane >> 2) * 8192 +
+                       (lane & 3) * 2048;
+        const CUtensorMap* m = is_v ? (wide ? &maps.v : &maps.v16) : (wide ? &maps.k : &maps.k16);
+#pragma unroll
+        for (int dh = 0; dh < Cf::kHalves; ++dh)
+          tma_load_2d(dst + dh * Cf::kKVHalf, m, &sh.kv_full[slot], dh * 64, it.row0 + mine * 64);
       }
     }
   }
@@ -257,10 +367,7 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
   constexpr int kK = D / 16;  // k-steps of Q K^T
   const int pairs = (g.C + 1) / 2;
   const int items = g.B * g.H * pairs;
-  const int nsteps = (topk + 1) / 2;
-  const bool odd = (topk & 1) != 0;  // last step has 64 keys
-  constexpr uint32_t kIdescQK128 = idesc_bf16_f32(64, 128, false, false);
-  constexpr uint32_t kIdescQK64 = idesc_bf16_f32(64, 64, false, false);
+  constexpr uint32_t kIdescQK = idesc_bf16_f32(64, 128, false, false);
   const uint32_t ring_base = smem_u32(sh.base + Cf::kRingOff);
   // Ring position kept as (slot, phase) and advanced incrementally; the K and
   // V descriptors of slot 0 are built once and a slot adds its byte offset / 16
@@ -276,6 +383,14 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
     const int qb = t & 1;
     if (!mbar_wait(&sh.q_full[qb], (t >> 1) & 1)) return fail(sh, status);
     tc_fence_after();
+    // steps and last-step chunks of both cubes (the producer's chunk counts)
+    int n[2], last[2];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int T = sh.chunks[2 * qb + c];
+      n[c] = (T + 7) / 8;
+      last[c] = T - 8 * (n[c] - 1);
+    }
     const uint32_t qa0 = smem_u32(sh.base + qb * 2 * Cf::kQBytes);
     const uint64_t qdesc0 = sdesc_sw128(qa0, 16, 1024);
     const uint64_t qdesc1 = sdesc_sw128(qa0 + Cf::kQBytes, 16, 1024);
@@ -295,7 +410,8 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
       if (!next_slot(slot)) return false;
       const uint64_t a0 = c == 0 ? qdesc0 : qdesc1;
       const uint64_t b0 = kdesc_base + (slot * Cf::kSlotBytes >> 4);
-      const uint32_t idesc = (odd && j == nsteps - 1) ? kIdescQK64 : kIdescQK128;
+      const int nc = j == (c ? n[1] : n[0]) - 1 ? (c ? last[1] : last[0]) : 8;
+      const uint32_t idesc = (kIdescQK & ~(0x3Fu << 17)) | (static_cast<uint32_t>(2 * nc) << 17);
       const uint32_t dS = tmem + (c == 0 ? Cf::kColS0 : Cf::kColS1);
 #pragma unroll
       for (int kk = 0; kk < kK; ++kk) {
@@ -318,28 +434,35 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
       const uint64_t v0 = vdesc_base + (slot * Cf::kSlotBytes >> 4);
       const uint32_t dO = tmem + (c == 0 ? Cf::kColO0 : Cf::kColO1);
       const uint32_t aP = tmem + (c == 0 ? Cf::kColS0 : Cf::kColS1);
+      const int nsteps = c ? n[1] : n[0];
+      const int nc = j == nsteps - 1 ? (c ? last[1] : last[0]) : 8;
       const uint32_t acc0 = j > 0 ? 1u : 0u;
       umma_ts(dO, aP, v0, Cf::kIdescPV, acc0);
+      if (nc == 8) {
 #pragma unroll
-      for (int kk = 1; kk < 4; ++kk) umma_ts(dO, aP + kk * 8, v0 + (kk * 2048 >> 4), Cf::kIdescPV, 1u);
-      if (!(odd && j == nsteps - 1)) {
-#pragma unroll
-        for (int kk = 4; kk < 8; ++kk) umma_ts(dO, aP + kk * 8, v0 + (kk * 2048 >> 4), Cf::kIdescPV, 1u);
+        for (int kk = 1; kk < 8; ++kk)
+          umma_ts(dO, aP + kk * 8, v0 + (kk * 2048 >> 4), Cf::kIdescPV, 1u);
+      } else {
+        for (int kk = 1; kk < nc; ++kk)
+          umma_ts(dO, aP + kk * 8, v0 + (kk * 2048 >> 4), Cf::kIdescPV, 1u);
       }
       umma_commit(&sh.kv_empty[slot]);
       if (j == nsteps - 1) umma_commit(&sh.o_full[c]);
       return true;
     };
     if (!qk(0, 0)) return fail(sh, status);
-    if (it.has_b && !qk(1, 0)) return fail(sh, status);
+    if (n[1] > 0 && !qk(1, 0)) return fail(sh, status);
     // No abort check inside the item: a failed role stops feeding this
     // thread, whose next bounded wait then ends the item.
-    for (int j = 0; j < nsteps; ++j) {
-      if (!pv(0, j)) return fail(sh, status);
-      if (j + 1 < nsteps && !qk(0, j + 1)) return fail(sh, status);
-      if (it.has_b) {
+    const int nmax = max(n[0], n[1]);
+    for (int j = 0; j < nmax; ++j) {
+      if (j < n[0]) {
+        if (!pv(0, j)) return fail(sh, status);
+        if (j + 1 < n[0] && !qk(0, j + 1)) return fail(sh, status);
+      }
+      if (j < n[1]) {
         if (!pv(1, j)) return fail(sh, status);
-        if (j + 1 < nsteps && !qk(1, j + 1)) return fail(sh, status);
+        if (j + 1 < n[1] && !qk(1, j + 1)) return fail(sh, status);
       }
     }
     umma_commit(&sh.q_empty[qb]);  // Q buffer free once this item's MMAs complete
@@ -350,7 +473,7 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
 template <int D, bool kTokenOut>
 __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c,
                            const int32_t* __restrict__ sel, int topk, const OutSpec os,
-                           int* status) {
+                           int* status, const int32_t* __restrict__ counts) {
   __nv_bfloat16* __restrict__ out = os.out;
   float* __restrict__ lse = os.lse;
   using Cf = Cfg<D>;
@@ -365,7 +488,6 @@ __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c
   const float sl2 = kLog2e * rsqrtf(static_cast<float>(D));
   const int pairs = (g.C + 1) / 2;
   const int items = g.B * g.H * pairs;
-  const int nsteps = (topk + 1) / 2;
   uint32_t s_phase = 0u, o_phase = 0u;
 
   for (int item = blockIdx.x; item < items; item += gridDim.x) {
@@ -376,25 +498,46 @@ __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c
     const int ni = cube_valid(g, i);
     const int32_t* list = sel + (static_cast<long long>(it.bh) * g.C + i) * topk;
     float m_ref = -INFINITY, l_part = 0.f;
-    int next_idx = hh < topk ? __ldg(&list[hh]) : -1;  // key cube of this half, step 0
-    for (int j = 0; j < nsteps; ++j) {
-      int jr = next_idx;
-      const int an = 2 * (j + 1) + hh;  // prefetch the next step's index
-      next_idx = (j + 1 < nsteps && an < topk) ? __ldg(&list[an]) : -1;
-      int nh = 0;
-      if (2 * j + hh < topk) {
-        jr = jr < 0 ? 0 : (jr >= g.C ? g.C - 1 : jr);
-        nh = cube_valid(g, jr);
+    const int W = count_wide(g, list, topk, lane, nullptr);
+    const int T = 3 * W + topk;  // 16-row key chunks of the cube
+    // list entries of this thread's four chunks (the half-step from chunk
+    // 8j + 4hh), fetched one step ahead
+    auto fetch = [&](int j, Ahead (&a)[4]) {
+      const int cb = 8 * j + 4 * hh;
+      const int kind = half_kind(cb, W, T);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) a[q] = fetch_entry(list, kind == 0 ? -1 : half_entry(cb, q, W, topk));
+    };
+    Ahead ahead[4];
+    fetch(0, ahead);
+    for (int j = 0; 8 * j < T; ++j) {
+      // valid key rows of this thread's four chunks, from the cube_count table
+      // (checked against the grid by the producer; a mismatch is reported as
+      // VSA_ERR_BAD_INDEX, and since counts only set masks, never addresses,
+      // it cannot make the kernel read or write out of bounds)
+      const bool wide = half_kind(8 * j + 4 * hh, W, T) == 1;
+      int vc[4];
+      if (wide) {
+        const int n = __ldg(&counts[cube_of(g, ahead[0])]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) vc[q] = min(16, max(0, n - 16 * q));
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int cq = cube_of(g, ahead[q]);
+          vc[q] = cq >= 0 ? __ldg(&counts[cq]) : 0;
+        }
       }
+      fetch(j + 1, ahead);
       if (!mbar_wait(&sh.s_full[c], s_phase)) return fail(sh, status);
       s_phase ^= 1u;
       tc_fence_after();
       uint32_t sv[64];
       tmem_ld_16x32bx2_x64(tS, sv);
-      if (nh < 64) {  // partial or absent key cube: mask its pad slots
+      if ((vc[0] & vc[1] & vc[2] & vc[3]) != 16) {  // mask pad and absent key rows
 #pragma unroll
         for (int e = 0; e < 64; ++e)
-          if (e >= nh) sv[e] = __float_as_uint(-INFINITY);
+          if ((e & 15) >= vc[e >> 4]) sv[e] = __float_as_uint(-INFINITY);
       }
       float mx8[8];
 #pragma unroll
@@ -517,8 +660,7 @@ __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c
 
 template <int D, bool kTokenOut>
 __global__ void __launch_bounds__(kThreads, 1) fine_fwd_kernel(
-    const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-    const __grid_constant__ CUtensorMap tv, Geom g, const int32_t* __restrict__ counts,
+    const __grid_constant__ FineMaps maps, Geom g, const int32_t* __restrict__ counts,
     const int32_t* __restrict__ sel, int topk, const OutSpec os, int* status) {
   using Cf = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -536,6 +678,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_fwd_kernel(
   sh.o_full = sh.s_full + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sh.o_full + 2);
   sh.abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  sh.chunks = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == kMmaWarp) {
@@ -556,9 +699,11 @@ __global__ void __launch_bounds__(kThreads, 1) fine_fwd_kernel(
     }
     *sh.abort_flag = 0;
     fence_barrier_init();
-    prefetch_tmap(&tq);
-    prefetch_tmap(&tk);
-    prefetch_tmap(&tv);
+    prefetch_tmap(&maps.q);
+    prefetch_tmap(&maps.k);
+    prefetch_tmap(&maps.v);
+    prefetch_tmap(&maps.k16);
+    prefetch_tmap(&maps.v16);
   }
   tc_fence_before();
   __syncthreads();
@@ -566,11 +711,11 @@ __global__ void __launch_bounds__(kThreads, 1) fine_fwd_kernel(
   const uint32_t tmem = *tmem_slot;
 
   if (warp == kProducerWarp) {
-    producer<D>(sh, g, &tq, &tk, &tv, counts, sel, topk, status);
+    producer<D>(sh, g, maps, counts, sel, topk, status);
   } else if (warp == kMmaWarp) {
     if (lane == 0) mma_issuer<D>(sh, g, tmem, topk, status);
   } else if (warp >= kSoftmaxWarp0) {
-    softmax_wg<D, kTokenOut>(sh, g, tmem, (warp - kSoftmaxWarp0) >> 2, sel, topk, os, status);
+    softmax_wg<D, kTokenOut>(sh, g, tmem, (warp - kSoftmaxWarp0) >> 2, sel, topk, os, status, counts);
   }
   tc_fence_before();
   __syncthreads();
@@ -581,8 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_fwd_kernel(
 
 size_t fine_smem_bytes(int d) { return d == 128 ? Cfg<128>::kSmem : Cfg<64>::kSmem; }
 
-cudaError_t launch_block_sparse_fwd(const Geom& g, const CUtensorMap& tq, const CUtensorMap& tk,
-                                    const CUtensorMap& tv, const int32_t* counts,
+cudaError_t launch_block_sparse_fwd(const Geom& g, const FineMaps& maps, const int32_t* counts,
                                     const int32_t* sel, int topk, void* out, float* lse,
                                     const float* o_coarse, const float* g_fine,
                                     const float* g_coarse, bool token_order, int* status, int sms,
@@ -598,7 +742,7 @@ cudaError_t launch_block_sparse_fwd(const Geom& g, const CUtensorMap& tq, const 
   auto run = [&](auto kernel, int which) -> cudaError_t {
     cudaError_t e = smem_limit_once(kernel, static_cast<int>(smem), &limit_set[which]);
     if (e != cudaSuccess) return e;
-    kernel<<<grid, kThreads, smem, s>>>(tq, tk, tv, g, counts, sel, topk, os, status);
+    kernel<<<grid, kThreads, smem, s>>>(maps, g, counts, sel, topk, os, status);
     return cudaSuccess;
   };
   if (g.d == 128)

@@ -1,0 +1,15 @@
+// Tensor maps the fine block-sparse kernel loads its tiles through.
+#pragma once
+
+#include <cuda.h>
+
+namespace vsa {
+
+// All over the tiled [B*H*64C rows, d] bf16 tensors, 128-byte swizzle,
+// 64-column boxes: q, k, v with 64-row boxes (one cube), k16, v16 with
+// 16-row boxes (the valid rows of a cube with at most 16 tokens).
+struct FineMaps {
+  CUtensorMap q, k, v, k16, v16;
+};
+
+}  // namespace vsa
