@@ -29,7 +29,7 @@ cudaError_t launch_block_sparse_fwd(const Geom&, const FineMaps&, const int32_t*
                                     bool, int*, int, cudaStream_t);
 cudaError_t launch_debug_wait(uint64_t, int*, cudaStream_t);
 cudaError_t launch_select_transpose(int, int, int, const int32_t*, int32_t*, int32_t*, int32_t*,
-                                    int*, cudaStream_t);
+                                    int*, int, cudaStream_t);
 cudaError_t launch_backward_prep(const Geom&, const void*, const void*, const float*, const float*,
                                  const float*, void*, float*, float*, float*, float*, cudaStream_t);
 cudaError_t launch_coarse_backward(int, int, int, const float*, const float*, const float*, float*,
@@ -432,7 +432,7 @@ int vsa_select_transpose(const vsa_shape* shape, const int32_t* sel_idx, int top
   DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_select_transpose(g.B * g.H, g.C, topk, sel_idx, key_offsets, query_lists,
-                                         static_cast<int32_t*>(workspace), st.status, stream));
+                                         static_cast<int32_t*>(workspace), st.status, st.sms, stream));
 }
 
 int vsa_backward_prep(const vsa_shape* shape, const void* dout, const void* o_fine_tiled,

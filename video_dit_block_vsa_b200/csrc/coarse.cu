@@ -109,7 +109,7 @@ constexpr int kTopkRegs = 48;
 // the others, each group in ascending order.  Executed by one full warp; hist
 // is a warp-private 256-entry smem array.  Most-significant-digit-first radix
 // select over the order-preserving integer image of the floats, 8 bits per
-// pass, then two ballot-compaction passes in index order.
+// pass, then one ballot-compaction pass in index order.
 __device__ void warp_topk(const Geom& g, const float* row, int C, int k, int* hist,
                           int32_t* out) {
   const int lane = threadIdx.x & 31;
@@ -171,42 +171,40 @@ __device__ void warp_topk(const Geom& g, const float* row, int C, int k, int* hi
     __syncwarp();
   }
   // prefix = key of the k-th largest; take all keys above it and the first
-  // `remaining` keys equal to it in index order.  The taken keys are written
-  // in two passes, the key cubes with more than 16 valid tokens first, then
-  // the others, each in ascending index order (the order the fine kernel
-  // packs key rows in); which keys are taken does not depend on the pass.
+  // `remaining` keys equal to it in index order.  One pass in index order
+  // writes the taken key cubes with more than 16 valid tokens from the front
+  // of out[] and the others from the back; reversing the back part then
+  // leaves both groups ascending, wide ones first (the order the fine kernel
+  // packs key rows in).
   const unsigned lt = (1u << lane) - 1u;
-  auto emit = [&](bool want_wide, int pos) -> int {
-    int eq_seen = 0;
-#pragma unroll
-    for (int u = 0; u < kTopkRegs; ++u) {
-      const int j = lane + 32 * u;
-      const bool gt = j < C && kc[u] > prefix;
-      const bool eq = j < C && kc[u] == prefix;
-      const unsigned eqm = __ballot_sync(0xffffffffu, eq);
-      const bool take = (gt || (eq && eq_seen + __popc(eqm & lt) < remaining)) &&
-                        ((cube_valid(g, j < C ? j : 0) > 16) == want_wide);
-      const unsigned tm = __ballot_sync(0xffffffffu, take);
-      if (take) out[pos + __popc(tm & lt)] = j;
-      pos += __popc(tm);
-      eq_seen += __popc(eqm);
-    }
-    for (int j0 = 32 * kTopkRegs; j0 < C; j0 += 32) {
-      const int j = j0 + lane;
-      const uint32_t key = j < C ? order_key(row[j]) : 0u;
-      const bool gt = j < C && key > prefix;
-      const bool eq = j < C && key == prefix;
-      const unsigned eqm = __ballot_sync(0xffffffffu, eq);
-      const bool take = (gt || (eq && eq_seen + __popc(eqm & lt) < remaining)) &&
-                        ((cube_valid(g, j < C ? j : 0) > 16) == want_wide);
-      const unsigned tm = __ballot_sync(0xffffffffu, take);
-      if (take) out[pos + __popc(tm & lt)] = j;
-      pos += __popc(tm);
-      eq_seen += __popc(eqm);
-    }
-    return pos;
+  int pos_w = 0, pos_n = 0, eq_seen = 0;
+  auto take_window = [&](int j, uint32_t key) {
+    const bool gt = j < C && key > prefix;
+    const bool eq = j < C && key == prefix;
+    const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && eq_seen + __popc(eqm & lt) < remaining);
+    const bool wide = cube_valid(g, j < C ? j : 0) > 16;
+    const unsigned wm = __ballot_sync(0xffffffffu, take && wide);
+    const unsigned nm = __ballot_sync(0xffffffffu, take && !wide);
+    if (take && wide) out[pos_w + __popc(wm & lt)] = j;
+    if (take && !wide) out[k - 1 - (pos_n + __popc(nm & lt))] = j;
+    pos_w += __popc(wm);
+    pos_n += __popc(nm);
+    eq_seen += __popc(eqm);
   };
-  emit(false, emit(true, 0));
+#pragma unroll
+  for (int u = 0; u < kTopkRegs; ++u) take_window(lane + 32 * u, kc[u]);
+  for (int j0 = 32 * kTopkRegs; j0 < C; j0 += 32) {
+    const int j = j0 + lane;
+    take_window(j, j < C ? order_key(row[j]) : 0u);
+  }
+  __syncwarp();
+  // out[pos_w .. k) holds the narrow cubes in descending order: reverse it
+  for (int a = lane; a < pos_n / 2; a += 32) {
+    const int x = out[pos_w + a], y = out[k - 1 - a];
+    out[pos_w + a] = y;
+    out[k - 1 - a] = x;
+  }
 }
 
 // ------------------------------------------------------------------ coarse
