@@ -25,6 +25,7 @@ from __future__ import annotations
 
 import argparse
 import csv
+import dataclasses
 import io
 import json
 import math
@@ -477,6 +478,7 @@ def run_backward_pieces(args, w):
     c_ws = torch.empty(vsa.vsa_coarse_backward_workspace_bytes(shape), dtype=torch.uint8, device=dev)
     pooled = vsa.pooled_view(shape, bufs.workspace)
     stream = torch.cuda.current_stream()
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
     pieces = {
         "backward_prep": lambda: vsa.vsa_backward_prep(shape, dout, bufs.o_f, dof, delta, bufs.o_c,
                                                        g_f, g_c, doc, dgf, dgc),
@@ -484,6 +486,9 @@ def run_backward_pieces(args, w):
                                                              t_ws),
         "coarse_backward": lambda: vsa.vsa_coarse_backward(shape, pooled, bufs.o_c, doc, d_pooled,
                                                            c_ws),
+        "fine_backward": lambda: vsa.vsa_block_sparse_bwd(shape, bufs.q_t, bufs.k_t, bufs.v_t,
+                                                          bufs.sel, w.topk, offs, lists, bufs.lse,
+                                                          dof, delta, dq, dk, dv, d_pooled),
     }
     ms = {}
     for name, fn in pieces.items():
@@ -509,6 +514,12 @@ def run_backward_pieces(args, w):
     # coarse backward: the 5 C x C x d products (S, dP, dQ, dK, dV) of a
     # backward, 2 flops each multiply-add
     coarse_flops = 10.0 * B * H * C * C * d
+    # fine backward: per (query cube, selected key cube) the products S, dP, dQ
+    # (query side) and S^T, dP^T, dK, dV (key side) over valid tokens only
+    counts = cube_counts(w.grid)
+    sel_np = bufs.sel.cpu().numpy().astype(np.int64)
+    pair_tokens = float(np.sum(counts[None, None, :] * counts[sel_np].sum(axis=-1)))
+    fine_bwd_flops = 14.0 * d * pair_tokens
     line = {"mode": "backward_pieces", "workload": w.name, "steps": args.steps,
             "warmup": args.warmup, "ms": {k_: round(v_, 4) for k_, v_ in ms.items()},
             "backward_prep": {"algorithmic_bytes": prep_bytes,
@@ -517,7 +528,91 @@ def run_backward_pieces(args, w):
                               "gated": True},
             "coarse_backward": {"algorithmic_flops": coarse_flops,
                                 "achieved_tflops": round(coarse_flops / ms["coarse_backward"] / 1e9, 2),
-                                "dtype": "f32", "note": "SIMT float32 register-tiled products"}}
+                                "dtype": "f32", "note": "SIMT float32 register-tiled products"},
+            "fine_backward": {"algorithmic_flops": fine_bwd_flops,
+                              "achieved_tflops": round(fine_bwd_flops / ms["fine_backward"] / 1e9, 2),
+                              "dtype": "bf16 in, f32 arithmetic",
+                              "note": "SIMT float32 register-tiled products; 7 products per block pair"}}
+    print(json.dumps(line))
+    return 0
+
+
+# float32 FMA lanes per SM of a B200 (4 sub-partitions x 32); the SIMT
+# products' ALU roofline is this x 2 flops x SMs x the sampled SM clock.
+FP32_LANES_PER_SM = 128
+
+
+def run_sparse_linear(args, w):
+    """Times the sparse + linear forward on the workload (one GPU, not the
+    default bench line): the three-launch block-sparse forward, then the
+    low-rank linear compensation branch added to its output in place.  The
+    branch's roofline is the float32 FMA peak (its products run on the SIMT
+    lanes).  Prints one JSON line."""
+    import torch
+
+    from video_dit_block_vsa_b200 import vsa
+
+    x = wl.make_inputs(w)
+    shape = vsa.make_shape(w.batch, w.heads, w.head_dim, w.grid)
+    dev = torch.device("cuda", 0)
+    to_dev = lambda b: torch.from_numpy(b.view(np.int16)).to(dev).view(torch.bfloat16)
+    q, k, v = to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"])
+    B, H, N, d = w.batch, w.heads, w.tokens, w.head_dim
+    g_f = torch.from_numpy(x["g_f"]).to(dev) if w.gated else None
+    g_c = torch.from_numpy(x["g_c"]).to(dev) if w.gated else None
+    out = torch.empty_like(q)
+    bufs = vsa.VsaBuffers(shape, w.topk, device=dev, want_coarse=w.gated)
+    ws = torch.empty(vsa.vsa_linear_workspace_bytes(shape), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def forward():
+        vsa.vsa_forward_fused(shape, q, k, v, w.topk, out, g_f, g_c, bufs=bufs)
+
+    def branch():
+        vsa.vsa_linear_branch_add(shape, q, k, v, out, ws)
+
+    def both():
+        forward()
+        branch()
+
+    sampler = ClockSampler(0)
+    clocks = None
+    ms = {}
+    for name, fn in (("sparse_forward", forward), ("linear_branch", branch), ("sparse_plus_linear", both)):
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        if name == "linear_branch":
+            sampler.start()
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if name == "linear_branch":
+            clocks = sampler.stop() or {}
+        ms[name] = a.elapsed_time(b) / args.steps
+    status = vsa.vsa_get_status()
+    if status != 0:
+        raise RuntimeError(f"device status: {vsa.vsa_strerror(status)}")
+    # KV = phi(K)^T V and phi(Q) KV: 2 N d^2 flops each; z and phi(Q) z: 2 N d each
+    flops = float(B * H) * (4.0 * N * d * d + 4.0 * N * d)
+    mhz = clocks.get("sm_mhz") or 1965.0
+    peak = 148 * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+    achieved = flops / ms["linear_branch"] / 1e9
+    # K, V read by the first pass, Q read and the output read and written by the last
+    bytes_ = float(B * H * N * d * 2) * 4
+    line = {"mode": "sparse_linear", "workload": w.name, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms": {k_: round(v_, 4) for k_, v_ in ms.items()},
+            "linear_branch": {"algorithmic_flops": flops, "achieved_tflops": round(achieved, 2),
+                              "bound": "alu", "peak_tflops": round(peak, 1),
+                              "peak_kind": "float32 FMA: 148 SMs x 128 lanes x 2 x sampled SM clock",
+                              "frac": round(achieved / peak, 4),
+                              "algorithmic_bytes": bytes_,
+                              "achieved_gbs": round(bytes_ / ms["linear_branch"] / 1e6, 1),
+                              "dtype": "bf16 in, f32 arithmetic"},
+            "clocks": clocks}
     print(json.dumps(line))
     return 0
 
@@ -538,10 +633,20 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward-pieces", action="store_true",
                     help="time the backward pieces built so far instead (one GPU)")
+    ap.add_argument("--sparse-linear", action="store_true",
+                    help="time the sparse + linear forward (block-sparse forward plus the low-rank "
+                         "linear branch) instead (one GPU)")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run the workload with fewer heads (small cases for profiler captures; "
+                         "the bench line's config names the heads)")
     args = ap.parse_args()
     w = wl.WORKLOADS[args.workload]
+    if args.heads is not None:
+        w = dataclasses.replace(w, heads=args.heads)
     if args.backward_pieces:
         return run_backward_pieces(args, w)
+    if args.sparse_linear:
+        return run_sparse_linear(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)

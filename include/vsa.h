@@ -240,6 +240,32 @@ int vsa_combine(const vsa_shape* shape, const void* o_fine_tiled, const float* o
  * pad rows are dropped. */
 int vsa_untile(const vsa_shape* shape, const void* x_tiled, void* x, cudaStream_t stream);
 
+/* Bytes of device workspace vsa_linear_branch_add needs for this shape
+ * (per-chunk partial sums and the per-(b, h) totals, float32), or 0 for an
+ * invalid shape. */
+size_t vsa_linear_workspace_bytes(const vsa_shape* shape);
+
+/* Low-rank linear compensation branch, added to an output in place (the
+ * sparse + linear variant: the SparkDiffusion page, RoLA paragraph, pairs a
+ * block-sparse branch with a low-rank linear branch that keeps the global
+ * context at 97 % sparsity; the TurboDiffusion review names trainable
+ * sparse-linear attention).  The pages print no formula; reading taken: for
+ * every token r of each (b, h) sequence,
+ *   out[r] += phi(q_r)^T KV / (phi(q_r)^T z),
+ *   KV = sum over all tokens t of phi(k_t) v_t^T,  z = sum_t phi(k_t),
+ * with phi(x) = elu(x) + 1 (positive, so the divisor never vanishes); the
+ * N x N attention matrix of this branch has rank at most d.  Run after the
+ * block-sparse forward (for example vsa_block_sparse_fwd_out) to get
+ * out = O_block_sparse + O_linear.  float32 arithmetic, fixed summation order
+ * (deterministic), the sum rounded to bf16.
+ *   q, k, v   bf16 [B, H, N, d] token order (read)
+ *   out       bf16 [B, H, N, d] token order (read and written)
+ *   workspace device scratch of at least vsa_linear_workspace_bytes(shape)
+ *             bytes, 256-byte aligned; contents on entry are ignored */
+int vsa_linear_branch_add(const vsa_shape* shape, const void* q, const void* k, const void* v,
+                          void* out, void* workspace, size_t workspace_bytes,
+                          cudaStream_t stream);
+
 /* Bytes of device workspace vsa_forward_host needs: two chunk buffers, each
  * holding heads_per_chunk (b, h) planes of the inputs, their tiled copies,
  * the final output and the coarse-stage scratch.  heads_per_chunk

@@ -28,6 +28,9 @@ cudaError_t launch_block_sparse_fwd(const Geom&, const FineMaps&, const int32_t*
                                     int, void*, float*, const float*, const float*, const float*,
                                     bool, int*, int, cudaStream_t);
 cudaError_t launch_debug_wait(uint64_t, int*, cudaStream_t);
+size_t linear_workspace_floats(int bh, long long N, int d);
+cudaError_t launch_linear_branch(int bh, long long N, int d, const void* q, const void* k,
+                                 const void* v, void* out, float* ws, cudaStream_t s);
 cudaError_t launch_select_transpose(int, int, int, const int32_t*, int32_t*, int32_t*, int32_t*,
                                     int*, int, cudaStream_t);
 cudaError_t launch_backward_prep(const Geom&, const void*, const void*, const float*, const float*,
@@ -249,6 +252,31 @@ int vsa_tile_permute(const vsa_shape* shape, const void* x, void* x_tiled, int32
   DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_tile_permute(g, x, x_tiled, cube_count, st.sms, stream));
+}
+
+size_t vsa_linear_workspace_bytes(const vsa_shape* shape) {
+  Geom g;
+  if (make_geom(shape, &g) != VSA_OK) return 0;
+  const size_t bytes = linear_workspace_floats(g.B * g.H, g.N, g.d) * sizeof(float);
+  return (bytes + 255) & ~static_cast<size_t>(255);
+}
+
+int vsa_linear_branch_add(const vsa_shape* shape, const void* q, const void* k, const void* v,
+                          void* out, void* workspace, size_t workspace_bytes,
+                          cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (!q || !k || !v || !out || !workspace || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      !aligned16(out) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < vsa_linear_workspace_bytes(shape))
+    return VSA_ERR_INVALID_ARG;
+  if (static_cast<long long>(g.B) * g.H > 65535 || (g.N + 63) / 64 > 0x7fffffffll)
+    return VSA_ERR_UNSUPPORTED;
+  DeviceState st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  return cuda_rc(launch_linear_branch(g.B * g.H, g.N, g.d, q, k, v, out,
+                                      static_cast<float*>(workspace), stream));
 }
 
 int vsa_untile(const vsa_shape* shape, const void* x_tiled, void* x, cudaStream_t stream) {

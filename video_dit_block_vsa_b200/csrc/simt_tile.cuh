@@ -78,13 +78,13 @@ __device__ __forceinline__ void stage_rows_t(float* dst, const T* __restrict__ s
 __device__ __forceinline__ int tile_col(int tx, int c) { return (c >> 2) * 64 + tx * 4 + (c & 3); }
 
 // acc[r][c] += sum over the chunk of As[k][ty*4 + r] * Bs[k][tile_col(tx, c)],
-// As with row stride kTileM, Bs with row stride BN.
+// As with row stride lda (kTileM unless given), Bs with row stride BN.
 template <int BN>
 __device__ __forceinline__ void chunk_fma(const float* As, const float* Bs, int tx, int ty,
-                                          float (&acc)[4][BN / 16]) {
+                                          float (&acc)[4][BN / 16], int lda = kTileM) {
 #pragma unroll 8
   for (int k = 0; k < kChunk; ++k) {
-    const float4 a = *reinterpret_cast<const float4*>(&As[k * kTileM + ty * 4]);
+    const float4 a = *reinterpret_cast<const float4*>(&As[k * lda + ty * 4]);
     const float av[4] = {a.x, a.y, a.z, a.w};
     float bv[BN / 16];
 #pragma unroll

@@ -37,7 +37,8 @@ EXPORTED = ("vsa_num_cubes", "vsa_topk_from_ratio", "vsa_workspace_bytes", "vsa_
             "vsa_block_sparse_fwd", "vsa_block_sparse_fwd_out",
             "vsa_combine", "vsa_untile", "vsa_forward_host_workspace_bytes", "vsa_forward_host",
             "vsa_select_transpose", "vsa_backward_prep", "vsa_coarse_backward_workspace_bytes", "vsa_coarse_backward",
-            "vsa_block_sparse_bwd", "vsa_get_status", "vsa_debug_wait_timeout",
+            "vsa_block_sparse_bwd", "vsa_linear_workspace_bytes", "vsa_linear_branch_add",
+            "vsa_get_status", "vsa_debug_wait_timeout",
             "vsa_strerror")
 
 
@@ -72,6 +73,8 @@ _sig = {
                                                 _P, _P, _P]),
     "vsa_combine": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, _P]),
     "vsa_untile": (ctypes.c_int, [_SP, _P, _P, _P]),
+    "vsa_linear_workspace_bytes": (ctypes.c_size_t, [_SP]),
+    "vsa_linear_branch_add": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "vsa_forward_host_workspace_bytes": (ctypes.c_size_t, [_SP, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "vsa_forward_host": (ctypes.c_int, [_SP, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                         ctypes.c_int, _P]),
@@ -324,6 +327,21 @@ def vsa_untile(shape, x_tiled, x, stream=None):
     _expect(x, torch.bfloat16, (B, H, N, d), "x")
     _check(_lib.vsa_untile(ctypes.byref(shape), _ptr(x_tiled), _ptr(x), _stream(stream)),
            "vsa_untile")
+
+
+def vsa_linear_workspace_bytes(shape) -> int:
+    return int(_lib.vsa_linear_workspace_bytes(ctypes.byref(shape)))
+
+
+def vsa_linear_branch_add(shape, q, k, v, out, workspace, stream=None):
+    """Adds the low-rank linear branch to ``out`` in place (see vsa.h)."""
+    B, H, N, d, C = _dims(shape)
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        _expect(t, torch.bfloat16, (B, H, N, d), n)
+    _expect_device(workspace, "workspace")
+    _check(_lib.vsa_linear_branch_add(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _stream(stream)), "vsa_linear_branch_add")
 
 
 def _expect_host(t, dtype, shape, name):
