@@ -520,6 +520,8 @@ def run_backward_pieces(args, w):
     sel_np = bufs.sel.cpu().numpy().astype(np.int64)
     pair_tokens = float(np.sum(counts[None, None, :] * counts[sel_np].sum(axis=-1)))
     fine_bwd_flops = 14.0 * d * pair_tokens
+    # issued: the 7 products run on whole 64 x 64 blocks
+    fine_bwd_issued = 14.0 * d * 64 * 64 * float(sel_np.size)
     line = {"mode": "backward_pieces", "workload": w.name, "steps": args.steps,
             "warmup": args.warmup, "ms": {k_: round(v_, 4) for k_, v_ in ms.items()},
             "backward_prep": {"algorithmic_bytes": prep_bytes,
@@ -531,8 +533,13 @@ def run_backward_pieces(args, w):
                                 "dtype": "f32", "note": "SIMT float32 register-tiled products"},
             "fine_backward": {"algorithmic_flops": fine_bwd_flops,
                               "achieved_tflops": round(fine_bwd_flops / ms["fine_backward"] / 1e9, 2),
-                              "dtype": "bf16 in, f32 arithmetic",
-                              "note": "SIMT float32 register-tiled products; 7 products per block pair"}}
+                              "issued_flops": fine_bwd_issued,
+                              "issued_tflops": round(fine_bwd_issued / ms["fine_backward"] / 1e9, 2),
+                              "peak_tflops": peaks["bf16"], "peak_source": peaks["source"],
+                              "frac": round(fine_bwd_flops / ms["fine_backward"] / 1e9 / peaks["bf16"], 4),
+                              "dtype": "bf16",
+                              "note": "tcgen05 (M = 64) products, float32 accumulation; 7 products "
+                                      "per block pair (S and dP in both the dq and the dk/dv kernel)"}}
     print(json.dumps(line))
     return 0
 

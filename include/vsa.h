@@ -369,10 +369,17 @@ int vsa_coarse_backward(const vsa_shape* shape, const float* pooled, const float
  *   d_pooled      float32 [3, B, H, C, d] from vsa_coarse_backward, or NULL
  *                 (ungated: the coarse output does not reach the result)
  *   dq, dk, dv    bf16 [B, H, N, d] token order (written, every token)
- * No atomics: one CTA per query cube accumulates dq over its key cubes, one
- * CTA per key cube accumulates dk, dv over the query cubes that selected it,
- * so the result is deterministic.  An index outside [0, C) in sel_idx or
- * query_lists is recorded as VSA_ERR_BAD_INDEX and skipped. */
+ * The products run on the tensor cores (tcgen05, bf16 operands, float32
+ * accumulation): P and dS are rounded to bf16 before they enter the dV, dQ
+ * and dK products, as in a bf16 training step.  No atomics: a query cube's
+ * dq is accumulated over its key cubes by one CTA, a key cube's dk, dv over
+ * the query cubes that selected it by one CTA, so the result is
+ * deterministic.  An index outside [0, C) in sel_idx or query_lists is
+ * recorded as VSA_ERR_BAD_INDEX and clamped into range; key_offsets that do
+ * not describe a list inside the CSR array are recorded the same way and the
+ * key cube is treated as selected by no query cube.  The tiled tensors, lse,
+ * delta, d_pooled and dq, dk, dv 16-byte aligned; on a wait that exceeds its
+ * bound the kernels record VSA_ERR_TIMEOUT and stop. */
 int vsa_block_sparse_bwd(const vsa_shape* shape, const void* q_tiled, const void* k_tiled,
                          const void* v_tiled, const int32_t* sel_idx, int topk,
                          const int32_t* key_offsets, const int32_t* query_lists, const float* lse,

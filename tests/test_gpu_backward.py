@@ -4,10 +4,12 @@ against the oracle's vsa_backward, which differentiates the float64 forward
 with the selection held at its choice.
 
 The GPU rounds where a bf16 training step would: O_f and the gated dO_f are
-bf16, P and dS float32, dq, dk, dv bf16.  A CPU emulation of those roundings
-lands within 4e-3 (max) and 2.4e-4 (mean) of the largest gradient on these
-cases; the bounds below leave 2.5x and 4x of room.  A wrong index, a
-transposed operand or a dropped term is off by the gradient's own size.
+bf16, P and dS are computed in float32 and enter the tensor-core products as
+bf16, the products accumulate in float32, dq, dk, dv are bf16.  A CPU
+emulation of those roundings lands within 5.6e-3 (max) and 3e-4 (mean) of
+the largest gradient on these cases; the bounds below leave 1.8x and 3x of
+room.  A wrong index, a transposed operand or a dropped term is off by the
+gradient's own size.
 
 """
 

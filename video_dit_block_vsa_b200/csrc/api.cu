@@ -38,10 +38,9 @@ cudaError_t launch_backward_prep(const Geom&, const void*, const void*, const fl
 cudaError_t launch_coarse_backward(int, int, int, const float*, const float*, const float*, float*,
                                    void*, size_t, cudaStream_t);
 size_t coarse_backward_plane_bytes(int C);
-cudaError_t launch_block_sparse_bwd(const Geom&, int, const void*, const void*, const void*,
-                                    const void*, const float*, const float*, const int32_t*,
-                                    const int32_t*, const int32_t*, const float*, void*, void*,
-                                    void*, int*, cudaStream_t);
+cudaError_t launch_block_sparse_bwd(const Geom&, const BwdMaps&, int, const float*, const float*,
+                                    const int32_t*, const int32_t*, const int32_t*, const float*,
+                                    void*, void*, void*, int*, int, cudaStream_t);
 
 // Device-side status word, one per device that loads the library.
 __device__ int g_status;
@@ -529,14 +528,17 @@ int vsa_block_sparse_bwd(const vsa_shape* shape, const void* q_tiled, const void
   if (!aligned16(q_tiled) || !aligned16(k_tiled) || !aligned16(v_tiled) ||
       !aligned16(do_fine_tiled) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
       (d_pooled && !aligned16(d_pooled)) || !a4(sel_idx) || !a4(key_offsets) ||
-      !a4(query_lists) || !a4(lse) || !a4(delta))
+      !a4(query_lists) || !aligned16(lse) || !aligned16(delta))
     return VSA_ERR_INVALID_ARG;
-  if (static_cast<long long>(g.B) * g.H > 65535) return VSA_ERR_UNSUPPORTED;  // grid y
   DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
-  return cuda_rc(launch_block_sparse_bwd(g, topk, q_tiled, k_tiled, v_tiled, do_fine_tiled, lse,
-                                         delta, sel_idx, key_offsets, query_lists, d_pooled, dq,
-                                         dk, dv, st.status, stream));
+  BwdMaps maps;
+  if (tiled_map(g, q_tiled, &maps.q) != VSA_OK || tiled_map(g, k_tiled, &maps.k) != VSA_OK ||
+      tiled_map(g, v_tiled, &maps.v) != VSA_OK || tiled_map(g, do_fine_tiled, &maps.dO) != VSA_OK)
+    return VSA_ERR_CUDA;
+  return cuda_rc(launch_block_sparse_bwd(g, maps, topk, lse, delta, sel_idx, key_offsets,
+                                         query_lists, d_pooled, dq, dk, dv, st.status, st.sms,
+                                         stream));
 }
 
 int vsa_get_status(cudaStream_t stream) {

@@ -1,4 +1,4 @@
-// Tensor maps the fine block-sparse kernel loads its tiles through.
+// Tensor maps the fine block-sparse kernels load their tiles through.
 #pragma once
 
 #include <cuda.h>
@@ -10,6 +10,12 @@ namespace vsa {
 // 16-row boxes (the valid rows of a cube with at most 16 tokens).
 struct FineMaps {
   CUtensorMap q, k, v, k16, v16;
+};
+
+// The fine backward's maps, 64-row boxes: tiled q, k, v and the tiled
+// gradient of the fine output (dO_f).
+struct BwdMaps {
+  CUtensorMap q, k, v, dO;
 };
 
 }  // namespace vsa
