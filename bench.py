@@ -626,7 +626,7 @@ def run_sparse_linear(args, w):
 
 # Revision tag of the fine kernel; ncu traffic figures are only reported for
 # the revision they were captured on.
-KERNEL_REV = "fine-v5-packed-out"
+KERNEL_REV = "fine-v6-static-producer-out"
 
 
 def main():

@@ -40,6 +40,8 @@
 //    VSA_ERR_TIMEOUT, every role stops, TMEM is freed and the CTA exits.
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "fine.cuh"
 #include "ptx.cuh"
@@ -158,12 +160,6 @@ __device__ __forceinline__ int half_entry(int cb, int q, int W, int topk) {
   if (cb < 4 * W) return q == 0 ? cb >> 2 : -1;
   const int e = W + (cb - 4 * W) + q;
   return e < topk ? e : -1;
-}
-
-// Key cube of list entry e (clamped into [0, C); the producer reports bad
-// entries), or -1 for e < 0.
-__device__ __forceinline__ int entry_cube(const Geom& g, const int32_t* list, int e) {
-  return e < 0 ? -1 : clamp_cube(g, __ldg(&list[e]));
 }
 
 // Wide entries of a list (warp-collective).  With `status`, also checks the
@@ -288,7 +284,10 @@ __device__ void producer(const Shared& sh, const Geom& g, const FineMaps& maps,
     // step j: V_Aj K_A(j+1) V_Bj K_B(j+1), skipping steps a cube does not have.
     // Lane q < 8 owns chunk slot q: its list entry for the next K load of each
     // cube is fetched one K load ahead, and a V load reuses the entries of the
-    // K load of the same step.
+    // K load of the same step.  Each cube's lookahead lives in its own
+    // variables and every slot is emitted by code specialised for its cube and
+    // kind, so no instruction that picks one cube's entry also waits for the
+    // other cube's load still in flight.
     auto lookup = [&](int c, int j) -> Ahead {
       const int Wc = c ? W[1] : W[0], Tc = c ? T[1] : T[0];
       const int cb = 8 * j + 4 * (lane >> 2);
@@ -296,48 +295,32 @@ __device__ void producer(const Shared& sh, const Geom& g, const FineMaps& maps,
       if (lane < 8 && half_kind(cb, Wc, Tc) != 0) e = half_entry(cb, lane & 3, Wc, topk);
       return fetch_entry(c ? list[1] : list[0], e);
     };
-    Ahead next_k[2] = {lookup(0, 0), lookup(1, 0)};
-    Ahead last_k[2] = {next_k[0], next_k[1]};
-    const int nmax = max(n[0], n[1]);
-    for (int e = 0;; ++e) {
-      int c, j;
-      bool is_v;
-      if (e < 2) {
-        c = e;
-        j = 0;
-        is_v = false;
-      } else {
-        const int js = (e - 2) >> 2, r = (e - 2) & 3;
-        if (js >= nmax) break;
-        c = r >> 1;
-        is_v = (r & 1) == 0;
-        j = is_v ? js : js + 1;
-      }
-      if (j >= (c ? n[1] : n[0])) continue;
-      if (*sh.abort_flag) return;
+    Ahead next_k0 = lookup(0, 0), next_k1 = lookup(1, 0);
+    Ahead last_k0 = next_k0, last_k1 = next_k1;
+    // one slot: 0 = issued, 1 = abort seen, 2 = a wait timed out
+    auto emit = [&](auto cube, auto value, int j) -> int {
+      constexpr int c = decltype(cube)::value;
+      constexpr bool is_v = decltype(value)::value;
+      Ahead& next_k = c ? next_k1 : next_k0;
+      Ahead& last_k = c ? last_k1 : last_k0;
+      if (*sh.abort_flag) return 1;
       const int slot = static_cast<int>(ring % Cf::kSlots);
       const uint32_t round = ring / Cf::kSlots;
       ++ring;
       // this step's chunk slots: lane q < 8 loads slot q's key cube
-      const int Wc = c ? W[1] : W[0], Tc = c ? T[1] : T[0];
+      const int Wc = W[c], Tc = T[c];
       const int cb0 = 8 * j;
       const bool wide = half_kind(cb0 + 4 * (lane >> 2), Wc, Tc) == 1;
       int mine;
-      if (is_v) {
-        mine = cube_of(g, c ? last_k[1] : last_k[0]);
+      if constexpr (is_v) {
+        mine = cube_of(g, last_k);
       } else {
-        const Ahead cur = c ? next_k[1] : next_k[0];
-        mine = cube_of(g, cur);
-        if (c) {
-          last_k[1] = cur;
-          next_k[1] = lookup(1, j + 1);
-        } else {
-          last_k[0] = cur;
-          next_k[0] = lookup(0, j + 1);
-        }
+        mine = cube_of(g, next_k);
+        last_k = next_k;
+        next_k = lookup(c, j + 1);
       }
       const int nc = min(8, Tc - cb0);
-      if (!wait_all(&sh.kv_empty[slot], (round & 1u) ^ 1u)) return fail(sh, status);
+      if (!wait_all(&sh.kv_empty[slot], (round & 1u) ^ 1u)) return 2;
       // the step's key rows: 64 per wide cube, 16 per narrow cube
       if (leader) mbar_arrive_expect_tx(&sh.kv_full[slot], static_cast<uint32_t>(nc) * 16u * D * 2u);
       __syncwarp();
@@ -349,7 +332,27 @@ __device__ void producer(const Shared& sh, const Geom& g, const FineMaps& maps,
         for (int dh = 0; dh < Cf::kHalves; ++dh)
           tma_load_2d(dst + dh * Cf::kKVHalf, m, &sh.kv_full[slot], dh * 64, it.row0 + mine * 64);
       }
+      return 0;
+    };
+    using A = std::integral_constant<int, 0>;
+    using B = std::integral_constant<int, 1>;
+    using K = std::false_type;
+    using V = std::true_type;
+    int rc = emit(A{}, K{}, 0);
+    if (rc == 0 && n[1] > 0) rc = emit(B{}, K{}, 0);
+    const int nmax = max(n[0], n[1]);
+    for (int js = 0; rc == 0 && js < nmax; ++js) {
+      if (js < n[0]) {
+        rc = emit(A{}, V{}, js);
+        if (rc == 0 && js + 1 < n[0]) rc = emit(A{}, K{}, js + 1);
+      }
+      if (rc == 0 && js < n[1]) {
+        rc = emit(B{}, V{}, js);
+        if (rc == 0 && js + 1 < n[1]) rc = emit(B{}, K{}, js + 1);
+      }
     }
+    if (rc == 1) return;
+    if (rc == 2) return fail(sh, status);
   }
 }
 
