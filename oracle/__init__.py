@@ -12,6 +12,9 @@ vsa_oracle : NumPy float64 restatement, stage by stage (tile permutation,
              attention, gated combine, untile).
 vsa_loops  : a second restatement with explicit Python loops and no BLAS, for
              tiny shapes only; it cross-checks ``vsa_oracle``.
+vsa_backward : gradients of the forward with the selection held fixed.
+vsa_linear : the low-rank linear compensation branch (sparse + linear).
+vsa_dit    : the QKV and output projections of a DiT block around VSA.
 
 Parity status per function is listed in each module's header.
 """
