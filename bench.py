@@ -624,6 +624,80 @@ def run_sparse_linear(args, w):
     return 0
 
 
+# Model width of the DiT block around the 720p workload (Wan-14B: 40 heads x 128).
+DIT_HIDDEN = {"wan14b_720p_21x45x80_k180": 5120, "wan14b_720p_21x45x80_k43": 5120,
+              "wan1.3b_ft_16x28x52": 1536, "wan1.3b_480p_21x30x52": 1536,
+              "scaling_16x32x32": 1536}
+
+
+def run_dit_block(args, w):
+    """Times a DiT attention block around VSA with the layout changes fused
+    into the projections (one GPU, not the default bench line): the QKV
+    projection writing q, k, v tiled, the coarse stage, the fine stage
+    (tiled output), and the output projection reading it tiled.  Random
+    weights of the model's width; prints one JSON line."""
+    import torch
+
+    from video_dit_block_vsa_b200 import vsa
+
+    hidden = DIT_HIDDEN.get(w.name, w.heads * w.head_dim)
+    B, H, N, d = w.batch, w.heads, w.tokens, w.head_dim
+    shape = vsa.make_shape(B, H, d, w.grid)
+    dev = torch.device("cuda", 0)
+    gen = torch.Generator(device=dev).manual_seed(w.seed)
+    x = torch.randn(B, N, hidden, device=dev, generator=gen).to(torch.bfloat16)
+    w_qkv = (torch.randn(3 * H * d, hidden, device=dev, generator=gen) * hidden ** -0.5).to(torch.bfloat16)
+    w_o = (torch.randn(hidden, H * d, device=dev, generator=gen) * (H * d) ** -0.5).to(torch.bfloat16)
+    y = torch.empty(B, N, hidden, dtype=torch.bfloat16, device=dev)
+    bufs = vsa.VsaBuffers(shape, w.topk, device=dev, want_coarse=False)
+    stream = torch.cuda.current_stream()
+    pieces = {
+        "qkv_projection_tiled": lambda: vsa.vsa_qkv_projection_tiled(
+            shape, hidden, x, w_qkv, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts),
+        "coarse_select": lambda: vsa.vsa_coarse_select(
+            shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, w.topk, bufs.sel, bufs.workspace),
+        "block_sparse_fwd": lambda: vsa.vsa_block_sparse_fwd(
+            shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, bufs.sel, w.topk, bufs.o_f),
+        "out_projection_tiled": lambda: vsa.vsa_out_projection_tiled(shape, hidden, bufs.o_f, w_o, y),
+    }
+    sampler = ClockSampler(0)
+    ms = {}
+    for name, fn in list(pieces.items()) + [("block", lambda: [f() for f in pieces.values()])]:
+        for _ in range(max(args.warmup, 3)):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        if name == "block":
+            sampler.start()
+        a.record(stream)
+        for _ in range(args.steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if name == "block":
+            clocks = sampler.stop() or {}
+        ms[name] = a.elapsed_time(b) / args.steps
+    status = vsa.vsa_get_status()
+    if status != 0:
+        raise RuntimeError(f"device status: {vsa.vsa_strerror(status)}")
+    peaks = load_peaks()
+    qkv_flops = 2.0 * B * N * hidden * 3 * H * d
+    out_flops = 2.0 * B * N * hidden * H * d
+    proj = {}
+    for name, fl in (("qkv_projection_tiled", qkv_flops), ("out_projection_tiled", out_flops)):
+        t = fl / ms[name] / 1e9
+        proj[name] = {"flops": fl, "achieved_tflops": round(t, 1), "peak_tflops": peaks["bf16"],
+                      "peak_source": peaks["source"], "frac": round(t / peaks["bf16"], 4)}
+    line = {"mode": "dit_block", "workload": w.name, "hidden": hidden, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms": {k_: round(v_, 4) for k_, v_ in ms.items()},
+            "projections": proj, "clocks": clocks,
+            "note": "tcgen05 GEMMs (128 x 256 tiles, bf16, float32 accumulation); the QKV "
+                    "projection writes q, k, v in the tiled layout and the output projection "
+                    "reads the tiled attention output and writes token order"}
+    print(json.dumps(line))
+    return 0
+
+
 # Revision tag of the fine kernel; ncu traffic figures are only reported for
 # the revision they were captured on.
 KERNEL_REV = "fine-v6-static-producer-out"
@@ -643,6 +717,9 @@ def main():
     ap.add_argument("--sparse-linear", action="store_true",
                     help="time the sparse + linear forward (block-sparse forward plus the low-rank "
                          "linear branch) instead (one GPU)")
+    ap.add_argument("--dit-block", action="store_true",
+                    help="time a DiT attention block with the projections fused around VSA instead "
+                         "(one GPU)")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload with fewer heads (small cases for profiler captures; "
                          "the bench line's config names the heads)")
@@ -654,6 +731,8 @@ def main():
         return run_backward_pieces(args, w)
     if args.sparse_linear:
         return run_sparse_linear(args, w)
+    if args.dit_block:
+        return run_dit_block(args, w)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)

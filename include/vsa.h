@@ -266,6 +266,40 @@ int vsa_linear_branch_add(const vsa_shape* shape, const void* q, const void* k, 
                           void* out, void* workspace, size_t workspace_bytes,
                           cudaStream_t stream);
 
+/* QKV projection of a DiT attention block with the tile permutation in its
+ * epilogue (FastWan news article, section "一张卡，秒生视频": VSA runs inside
+ * whole DiT blocks, between the QKV and the output projection; the pages give
+ * no formula, reading: the linear-layer convention, no bias):
+ *   [q | k | v] = x W_qkv^T, the 3 H d output features ordered q heads, k
+ *   heads, v heads (head h = features h d .. h d + d - 1),
+ * written straight into the tiled layout vsa_tile_permute produces (pad rows
+ * zero), plus the cube counts; bf16 operands, float32 accumulation on the
+ * tensor cores, bf16 results.
+ *   hidden        input features, a positive multiple of 64
+ *   x             bf16 [B, N, hidden] token order (read)
+ *   w_qkv         bf16 [3*H*d, hidden] (read)
+ *   q/k/v_tiled   bf16 [B, H, 64*C, d] (written, pad rows included)
+ *   cube_count    int32 [C] (written) or NULL
+ * Pointers 16-byte aligned.  On a wait that exceeds its bound the kernel
+ * records VSA_ERR_TIMEOUT and stops. */
+int vsa_qkv_projection_tiled(const vsa_shape* shape, int hidden, const void* x, const void* w_qkv,
+                             void* q_tiled, void* k_tiled, void* v_tiled, int32_t* cube_count,
+                             cudaStream_t stream);
+
+/* Output projection of a DiT attention block reading the attention output in
+ * the tiled layout, with the untile step in its epilogue:
+ *   y[b, n] = concat over heads h of o[b, h, n] times W_o^T
+ * where o[b, h, n] is the tiled row of token n (pad rows are read but never
+ * written anywhere).
+ *   hidden    output features, a positive multiple of 64
+ *   o_tiled   bf16 [B, H, 64*C, d], e.g. vsa_block_sparse_fwd's or
+ *             vsa_combine's output (read)
+ *   w_o       bf16 [hidden, H*d] (read)
+ *   y         bf16 [B, N, hidden] token order (written)
+ * Pointers 16-byte aligned. */
+int vsa_out_projection_tiled(const vsa_shape* shape, int hidden, const void* o_tiled,
+                             const void* w_o, void* y, cudaStream_t stream);
+
 /* Bytes of device workspace vsa_forward_host needs: two chunk buffers, each
  * holding heads_per_chunk (b, h) planes of the inputs, their tiled copies,
  * the final output and the coarse-stage scratch.  heads_per_chunk

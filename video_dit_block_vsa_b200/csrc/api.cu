@@ -31,6 +31,8 @@ cudaError_t launch_debug_wait(uint64_t, int*, cudaStream_t);
 size_t linear_workspace_floats(int bh, long long N, int d);
 cudaError_t launch_linear_branch(int bh, long long N, int d, const void* q, const void* k,
                                  const void* v, void* out, float* ws, cudaStream_t s);
+cudaError_t launch_projection(const Geom&, int, int, const CUtensorMap&, const CUtensorMap&, void*,
+                              void*, void*, int32_t*, int*, int, cudaStream_t);
 cudaError_t launch_select_transpose(int, int, int, const int32_t*, int32_t*, int32_t*, int32_t*,
                                     int*, int, cudaStream_t);
 cudaError_t launch_backward_prep(const Geom&, const void*, const void*, const float*, const float*,
@@ -276,6 +278,63 @@ int vsa_linear_branch_add(const vsa_shape* shape, const void* q, const void* k, 
   if ((rc = device_state(&st)) != VSA_OK) return rc;
   return cuda_rc(launch_linear_branch(g.B * g.H, g.N, g.d, q, k, v, out,
                                       static_cast<float*>(workspace), stream));
+}
+
+// A row-major bf16 matrix [rows, cols] with 128-byte-swizzled boxes of
+// 64 columns x box_rows rows.
+int matrix_map(const void* ptr, long long rows, long long cols, int box_rows, CUtensorMap* m) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;
+}
+
+int vsa_qkv_projection_tiled(const vsa_shape* shape, int hidden, const void* x, const void* w_qkv,
+                             void* q_tiled, void* k_tiled, void* v_tiled, int32_t* cube_count,
+                             cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (hidden < 64 || hidden % 64 != 0 || !x || !w_qkv || !q_tiled || !k_tiled || !v_tiled ||
+      !aligned16(x) || !aligned16(w_qkv) || !aligned16(q_tiled) || !aligned16(k_tiled) ||
+      !aligned16(v_tiled) || (cube_count && (reinterpret_cast<uintptr_t>(cube_count) & 3u)))
+    return VSA_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(g.B) * g.N;
+  if (rows >= (1ll << 31) || static_cast<long long>(hidden) * 3 * g.H * g.d >= (1ll << 40))
+    return VSA_ERR_UNSUPPORTED;
+  DeviceState st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  if ((rc = get_encoder()) != VSA_OK) return rc;
+  CUtensorMap amap, bmap;
+  if (matrix_map(x, rows, hidden, 128, &amap) != VSA_OK ||
+      matrix_map(w_qkv, 3ll * g.H * g.d, hidden, 256, &bmap) != VSA_OK)
+    return VSA_ERR_CUDA;
+  return cuda_rc(launch_projection(g, 0, hidden, amap, bmap, q_tiled, k_tiled, v_tiled, cube_count,
+                                   st.status, st.sms, stream));
+}
+
+int vsa_out_projection_tiled(const vsa_shape* shape, int hidden, const void* o_tiled,
+                             const void* w_o, void* y, cudaStream_t stream) {
+  Geom g;
+  int rc = make_geom(shape, &g);
+  if (rc != VSA_OK) return rc;
+  if (hidden < 64 || hidden % 64 != 0 || !o_tiled || !w_o || !y || !aligned16(o_tiled) ||
+      !aligned16(w_o) || !aligned16(y))
+    return VSA_ERR_INVALID_ARG;
+  DeviceState st;
+  if ((rc = device_state(&st)) != VSA_OK) return rc;
+  if ((rc = get_encoder()) != VSA_OK) return rc;
+  CUtensorMap amap, bmap;
+  if (matrix_map(o_tiled, static_cast<long long>(g.B) * g.H * g.rows, g.d, 128, &amap) != VSA_OK ||
+      matrix_map(w_o, hidden, static_cast<long long>(g.H) * g.d, 256, &bmap) != VSA_OK)
+    return VSA_ERR_CUDA;
+  return cuda_rc(launch_projection(g, 1, hidden, amap, bmap, y, nullptr, nullptr, nullptr,
+                                   st.status, st.sms, stream));
 }
 
 int vsa_untile(const vsa_shape* shape, const void* x_tiled, void* x, cudaStream_t stream) {
@@ -532,6 +591,7 @@ int vsa_block_sparse_bwd(const vsa_shape* shape, const void* q_tiled, const void
     return VSA_ERR_INVALID_ARG;
   DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
+  if ((rc = get_encoder()) != VSA_OK) return rc;
   BwdMaps maps;
   if (tiled_map(g, q_tiled, &maps.q) != VSA_OK || tiled_map(g, k_tiled, &maps.k) != VSA_OK ||
       tiled_map(g, v_tiled, &maps.v) != VSA_OK || tiled_map(g, do_fine_tiled, &maps.dO) != VSA_OK)

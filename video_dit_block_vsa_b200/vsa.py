@@ -38,6 +38,7 @@ EXPORTED = ("vsa_num_cubes", "vsa_topk_from_ratio", "vsa_workspace_bytes", "vsa_
             "vsa_combine", "vsa_untile", "vsa_forward_host_workspace_bytes", "vsa_forward_host",
             "vsa_select_transpose", "vsa_backward_prep", "vsa_coarse_backward_workspace_bytes", "vsa_coarse_backward",
             "vsa_block_sparse_bwd", "vsa_linear_workspace_bytes", "vsa_linear_branch_add",
+            "vsa_qkv_projection_tiled", "vsa_out_projection_tiled",
             "vsa_get_status", "vsa_debug_wait_timeout",
             "vsa_strerror")
 
@@ -75,6 +76,8 @@ _sig = {
     "vsa_untile": (ctypes.c_int, [_SP, _P, _P, _P]),
     "vsa_linear_workspace_bytes": (ctypes.c_size_t, [_SP]),
     "vsa_linear_branch_add": (ctypes.c_int, [_SP, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "vsa_qkv_projection_tiled": (ctypes.c_int, [_SP, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P]),
+    "vsa_out_projection_tiled": (ctypes.c_int, [_SP, ctypes.c_int, _P, _P, _P, _P]),
     "vsa_forward_host_workspace_bytes": (ctypes.c_size_t, [_SP, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "vsa_forward_host": (ctypes.c_int, [_SP, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                         ctypes.c_int, _P]),
@@ -342,6 +345,54 @@ def vsa_linear_branch_add(shape, q, k, v, out, workspace, stream=None):
     _check(_lib.vsa_linear_branch_add(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
                                       _stream(stream)), "vsa_linear_branch_add")
+
+
+def vsa_qkv_projection_tiled(shape, hidden, x, w_qkv, q_t, k_t, v_t, counts=None, stream=None):
+    """[q | k | v] = x W_qkv^T written straight into the tiled layout (see vsa.h)."""
+    B, H, N, d, C = _dims(shape)
+    _expect(x, torch.bfloat16, (B, N, hidden), "x")
+    _expect(w_qkv, torch.bfloat16, (3 * H * d, hidden), "w_qkv")
+    for n, t in (("q_t", q_t), ("k_t", k_t), ("v_t", v_t)):
+        _expect(t, torch.bfloat16, (B, H, 64 * C, d), n)
+    if counts is not None:
+        _expect(counts, torch.int32, (C,), "counts")
+    _check(_lib.vsa_qkv_projection_tiled(ctypes.byref(shape), int(hidden), _ptr(x), _ptr(w_qkv),
+                                         _ptr(q_t), _ptr(k_t), _ptr(v_t), _ptr(counts),
+                                         _stream(stream)), "vsa_qkv_projection_tiled")
+
+
+def vsa_out_projection_tiled(shape, hidden, o_t, w_o, y, stream=None):
+    """y = o W_o^T from the tiled attention output, written in token order (see vsa.h)."""
+    B, H, N, d, C = _dims(shape)
+    _expect(o_t, torch.bfloat16, (B, H, 64 * C, d), "o_t")
+    _expect(w_o, torch.bfloat16, (hidden, H * d), "w_o")
+    _expect(y, torch.bfloat16, (B, N, hidden), "y")
+    _check(_lib.vsa_out_projection_tiled(ctypes.byref(shape), int(hidden), _ptr(o_t), _ptr(w_o),
+                                         _ptr(y), _stream(stream)), "vsa_out_projection_tiled")
+
+
+def vsa_attention_block(shape, hidden, x, w_qkv, w_o, topk, y, g_fine=None, g_coarse=None,
+                        bufs=None, stream=None):
+    """A DiT attention block around VSA with the layout changes fused into the
+    projections: the QKV projection writes q, k, v tiled (and the cube
+    counts), the coarse stage pools them, the fine stage writes its output
+    tiled (combined with the coarse output when gated), and the output
+    projection reads it tiled and writes ``y`` in token order.  Returns the
+    buffers."""
+    if bufs is None:
+        bufs = VsaBuffers(shape, topk, device=x.device, want_coarse=g_fine is not None)
+    vsa_qkv_projection_tiled(shape, hidden, x, w_qkv, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts,
+                             stream)
+    vsa_coarse_select(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, topk, bufs.sel,
+                      bufs.workspace, o_coarse=bufs.o_c, stream=stream)
+    vsa_block_sparse_fwd(shape, bufs.q_t, bufs.k_t, bufs.v_t, bufs.counts, bufs.sel, topk,
+                         bufs.o_f, stream=stream)
+    o = bufs.o_f
+    if g_fine is not None:
+        vsa_combine(shape, bufs.o_f, bufs.out_t, bufs.o_c, g_fine, g_coarse, stream=stream)
+        o = bufs.out_t
+    vsa_out_projection_tiled(shape, hidden, o, w_o, y, stream)
+    return bufs
 
 
 def _expect_host(t, dtype, shape, name):
