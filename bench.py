@@ -544,17 +544,13 @@ def run_backward_pieces(args, w):
     return 0
 
 
-# float32 FMA lanes per SM of a B200 (4 sub-partitions x 32); the SIMT
-# products' ALU roofline is this x 2 flops x SMs x the sampled SM clock.
-FP32_LANES_PER_SM = 128
-
-
 def run_sparse_linear(args, w):
     """Times the sparse + linear forward on the workload (one GPU, not the
     default bench line): the three-launch block-sparse forward, then the
     low-rank linear compensation branch added to its output in place.  The
-    branch's roofline is the float32 FMA peak (its products run on the SIMT
-    lanes).  Prints one JSON line."""
+    branch moves little data per flop (two d x d products per token), so its
+    roofline is HBM: q, k, v read once and the output read and written.
+    Prints one JSON line."""
     import torch
 
     from video_dit_block_vsa_b200 import vsa
@@ -605,20 +601,22 @@ def run_sparse_linear(args, w):
         raise RuntimeError(f"device status: {vsa.vsa_strerror(status)}")
     # KV = phi(K)^T V and phi(Q) KV: 2 N d^2 flops each; z and phi(Q) z: 2 N d each
     flops = float(B * H) * (4.0 * N * d * d + 4.0 * N * d)
-    mhz = clocks.get("sm_mhz") or 1965.0
-    peak = 148 * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
-    achieved = flops / ms["linear_branch"] / 1e9
-    # K, V read by the first pass, Q read and the output read and written by the last
-    bytes_ = float(B * H * N * d * 2) * 4
+    # compulsory HBM bytes: q, k, v read once, the output read and written
+    bytes_ = float(B * H * N * d * 2) * 5
+    achieved_gbs = bytes_ / ms["linear_branch"] / 1e6
+    peaks = load_peaks()
     line = {"mode": "sparse_linear", "workload": w.name, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms": {k_: round(v_, 4) for k_, v_ in ms.items()},
-            "linear_branch": {"algorithmic_flops": flops, "achieved_tflops": round(achieved, 2),
-                              "bound": "alu", "peak_tflops": round(peak, 1),
-                              "peak_kind": "float32 FMA: 148 SMs x 128 lanes x 2 x sampled SM clock",
-                              "frac": round(achieved / peak, 4),
-                              "algorithmic_bytes": bytes_,
-                              "achieved_gbs": round(bytes_ / ms["linear_branch"] / 1e6, 1),
-                              "dtype": "bf16 in, f32 arithmetic"},
+            "linear_branch": {"bound": "hbm", "algorithmic_bytes": bytes_,
+                              "achieved_gbs": round(achieved_gbs, 1), "peak_gbs": peaks["hbm"],
+                              "peak_source": peaks["source"],
+                              "frac": round(achieved_gbs / peaks["hbm"], 4),
+                              "algorithmic_flops": flops,
+                              "achieved_tflops": round(flops / ms["linear_branch"] / 1e9, 2),
+                              "dtype": "bf16",
+                              "note": "phi(q), phi(k) written to and read back from the "
+                                      "workspace (bf16) by a separate pass; tcgen05 products "
+                                      "with float32 accumulation"},
             "clocks": clocks}
     print(json.dumps(line))
     return 0

@@ -241,8 +241,8 @@ int vsa_combine(const vsa_shape* shape, const void* o_fine_tiled, const float* o
 int vsa_untile(const vsa_shape* shape, const void* x_tiled, void* x, cudaStream_t stream);
 
 /* Bytes of device workspace vsa_linear_branch_add needs for this shape
- * (per-chunk partial sums and the per-(b, h) totals, float32), or 0 for an
- * invalid shape. */
+ * (phi(q) and phi(k) as bf16, per-chunk float32 partial sums of KV and z, and
+ * the bf16 [KV^T ; z^T] matrix of every (b, h)), or 0 for an invalid shape. */
 size_t vsa_linear_workspace_bytes(const vsa_shape* shape);
 
 /* Low-rank linear compensation branch, added to an output in place (the
@@ -256,8 +256,11 @@ size_t vsa_linear_workspace_bytes(const vsa_shape* shape);
  * with phi(x) = elu(x) + 1 (positive, so the divisor never vanishes); the
  * N x N attention matrix of this branch has rank at most d.  Run after the
  * block-sparse forward (for example vsa_block_sparse_fwd_out) to get
- * out = O_block_sparse + O_linear.  float32 arithmetic, fixed summation order
- * (deterministic), the sum rounded to bf16.
+ * out = O_block_sparse + O_linear.  The two products run on the tensor cores
+ * with bf16 operands (phi(q), phi(k), KV and z rounded to bf16) and float32
+ * accumulation, in a fixed summation order (deterministic); the sum is
+ * rounded to bf16.  On a wait that exceeds its bound the kernels record
+ * VSA_ERR_TIMEOUT and stop.
  *   q, k, v   bf16 [B, H, N, d] token order (read)
  *   out       bf16 [B, H, N, d] token order (read and written)
  *   workspace device scratch of at least vsa_linear_workspace_bytes(shape)

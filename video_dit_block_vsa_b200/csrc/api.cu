@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "fine.cuh"
+#include "linear.cuh"
 
 namespace vsa {
 
@@ -28,9 +29,11 @@ cudaError_t launch_block_sparse_fwd(const Geom&, const FineMaps&, const int32_t*
                                     int, void*, float*, const float*, const float*, const float*,
                                     bool, int*, int, cudaStream_t);
 cudaError_t launch_debug_wait(uint64_t, int*, cudaStream_t);
-size_t linear_workspace_floats(int bh, long long N, int d);
 cudaError_t launch_linear_branch(int bh, long long N, int d, const void* q, const void* k,
-                                 const void* v, void* out, float* ws, cudaStream_t s);
+                                 void* out, uint8_t* ws, const LinearLayout& L,
+                                 const CUtensorMap& fk_map, const CUtensorMap& v_map,
+                                 const CUtensorMap& fq_map, const CUtensorMap& b_map, int* status,
+                                 int sms, cudaStream_t s);
 cudaError_t launch_projection(const Geom&, int, int, const CUtensorMap&, const CUtensorMap&, void*,
                               void*, void*, int32_t*, int*, int, cudaStream_t);
 cudaError_t launch_select_transpose(int, int, int, const int32_t*, int32_t*, int32_t*, int32_t*,
@@ -258,9 +261,27 @@ int vsa_tile_permute(const vsa_shape* shape, const void* x, void* x_tiled, int32
 size_t vsa_linear_workspace_bytes(const vsa_shape* shape) {
   Geom g;
   if (make_geom(shape, &g) != VSA_OK) return 0;
-  const size_t bytes = linear_workspace_floats(g.B * g.H, g.N, g.d) * sizeof(float);
-  return (bytes + 255) & ~static_cast<size_t>(255);
+  return linear_layout(g.B * g.H, g.N, g.d).bytes;
 }
+
+// A bf16 tensor [planes][rows][cols] (cols contiguous) with 128-byte-swizzled
+// boxes of 64 columns x box_rows rows x 1 plane.
+int planes_map(const void* ptr, long long planes, long long rows, int cols, int box_rows,
+               CUtensorMap* m) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(planes)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2,
+                                 static_cast<cuuint64_t>(rows) * cols * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? VSA_OK : VSA_ERR_CUDA;
+}
+
+int matrix_map(const void* ptr, long long rows, long long cols, int box_rows, CUtensorMap* m);
 
 int vsa_linear_branch_add(const vsa_shape* shape, const void* q, const void* k, const void* v,
                           void* out, void* workspace, size_t workspace_bytes,
@@ -272,12 +293,20 @@ int vsa_linear_branch_add(const vsa_shape* shape, const void* q, const void* k, 
       !aligned16(out) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
       workspace_bytes < vsa_linear_workspace_bytes(shape))
     return VSA_ERR_INVALID_ARG;
-  if (static_cast<long long>(g.B) * g.H > 65535 || (g.N + 63) / 64 > 0x7fffffffll)
-    return VSA_ERR_UNSUPPORTED;
   DeviceState st;
   if ((rc = device_state(&st)) != VSA_OK) return rc;
-  return cuda_rc(launch_linear_branch(g.B * g.H, g.N, g.d, q, k, v, out,
-                                      static_cast<float*>(workspace), stream));
+  if ((rc = get_encoder()) != VSA_OK) return rc;
+  const int bh = g.B * g.H;
+  const LinearLayout L = linear_layout(bh, g.N, g.d);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  CUtensorMap fk_map, v_map, fq_map, b_map;
+  if (planes_map(ws + L.fk, bh, g.N, g.d, 64, &fk_map) != VSA_OK ||
+      planes_map(v, bh, g.N, g.d, 64, &v_map) != VSA_OK ||
+      planes_map(ws + L.fq, bh, g.N, g.d, 128, &fq_map) != VSA_OK ||
+      matrix_map(ws + L.bmat, static_cast<long long>(bh) * (g.d + 16), g.d, g.d + 16, &b_map) != VSA_OK)
+    return VSA_ERR_CUDA;
+  return cuda_rc(launch_linear_branch(bh, g.N, g.d, q, k, out, ws, L, fk_map, v_map, fq_map, b_map,
+                                      st.status, st.sms, stream));
 }
 
 // A row-major bf16 matrix [rows, cols] with 128-byte-swizzled boxes of
