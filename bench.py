@@ -327,7 +327,7 @@ def run_gpu(args, w):
     hgf = g_f.cpu().pin_memory() if w.gated else None
     hgc = g_c.cpu().pin_memory() if w.gated else None
     hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    chunk = HOST_CHUNK_HEADS
+    chunk = args.host_chunk_heads
     hws = torch.empty(vsa.vsa_forward_host_workspace_bytes(shape, w.topk, chunk, w.gated),
                       dtype=torch.uint8, device=dev)
 
@@ -718,6 +718,8 @@ def main():
     ap.add_argument("--dit-block", action="store_true",
                     help="time a DiT attention block with the projections fused around VSA instead "
                          "(one GPU)")
+    ap.add_argument("--host-chunk-heads", type=int, default=HOST_CHUNK_HEADS,
+                    help="(b, h) planes per chunk of the host-buffer path in the end-to-end leg")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload with fewer heads (small cases for profiler captures; "
                          "the bench line's config names the heads)")

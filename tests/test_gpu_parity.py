@@ -403,6 +403,13 @@ def check_workload(vsa, w, head_sample=None, cube_sample=None):
         assert_close(got[toks], ref[toks], f"{w.name} out (b={b}, h={h})")
 
 
+def test_largest_cube_count(vsa):
+    """C = 8192 cubes, the most a coarse row holds (32 x 128 x 128 latents, one
+    head, d = 64): the whole path against the oracle, selection on every row."""
+    w = wl.Workload("max_cubes_32x128x128", 1, 1, 64, (32, 128, 128), 8, 41, 0.5, False)
+    check_workload(vsa, w, cube_sample=12)
+
+
 @pytest.mark.parametrize("name", ["tiny_k2", "tiny_dense"])
 def test_workload_tiny_full(vsa, name):
     check_workload(vsa, wl.WORKLOADS[name])

@@ -70,6 +70,11 @@ def test_unsupported_shapes_rejected_before_launch(vsa):
     bad_b = vsa.make_shape(0, 1, 128, (8, 8, 8))
     assert lib.vsa_num_cubes(ctypes.byref(bad_b), ctypes.byref(c)) == vsa.VSA_ERR_INVALID_ARG
     assert lib.vsa_num_cubes(None, ctypes.byref(c)) == vsa.VSA_ERR_INVALID_ARG
+    # the most cubes a coarse row holds: 8192 accepted, more rejected
+    at_max = vsa.make_shape(1, 1, 64, (32, 128, 128))
+    assert lib.vsa_num_cubes(ctypes.byref(at_max), ctypes.byref(c)) == 0 and c.value == 8192
+    too_many = vsa.make_shape(1, 1, 64, (36, 128, 128))
+    assert lib.vsa_num_cubes(ctypes.byref(too_many), ctypes.byref(c)) == vsa.VSA_ERR_UNSUPPORTED
 
 
 def test_null_and_misaligned_pointers_rejected_before_launch(vsa):
@@ -137,6 +142,24 @@ def test_null_and_misaligned_pointers_rejected_before_launch(vsa):
     assert fb(ctypes.byref(s), p, p, p, p, 2, p, p, two, p, p, None, p, p, p, None) == vsa.VSA_ERR_INVALID_ARG
     assert fb(ctypes.byref(s), p, p, p, p, 2, p, p, p, p, p, odd, p, p, p, None) == vsa.VSA_ERR_INVALID_ARG
     assert lib.vsa_debug_wait_timeout(10, None) == vsa.VSA_ERR_INVALID_ARG
+    # linear branch: small or misaligned workspace, misaligned tensors
+    lb = lib.vsa_linear_branch_add
+    need = vsa.vsa_linear_workspace_bytes(s)
+    assert need > 0
+    ws = ctypes.c_void_p(0x100000)
+    assert lb(ctypes.byref(s), p, p, p, p, ws, need - 1, None) == vsa.VSA_ERR_INVALID_ARG
+    assert lb(ctypes.byref(s), p, p, p, p, ctypes.c_void_p(0x100010), need, None) == vsa.VSA_ERR_INVALID_ARG
+    assert lb(ctypes.byref(s), p, odd, p, p, ws, need, None) == vsa.VSA_ERR_INVALID_ARG
+    # projections: hidden must be a positive multiple of 64; pointers checked
+    qp, op_ = lib.vsa_qkv_projection_tiled, lib.vsa_out_projection_tiled
+    assert qp(ctypes.byref(s), 96, p, p, p, p, p, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert qp(ctypes.byref(s), 0, p, p, p, p, p, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert qp(ctypes.byref(s), 128, p, None, p, p, p, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert qp(ctypes.byref(s), 128, odd, p, p, p, p, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert qp(ctypes.byref(s), 128, p, p, p, p, p, two, None) == vsa.VSA_ERR_INVALID_ARG
+    assert op_(ctypes.byref(s), 96, p, p, p, None) == vsa.VSA_ERR_INVALID_ARG
+    assert op_(ctypes.byref(s), 128, p, p, None, None) == vsa.VSA_ERR_INVALID_ARG
+    assert op_(ctypes.byref(s), 128, p, odd, p, None) == vsa.VSA_ERR_INVALID_ARG
 
 
 def test_strerror(vsa):
