@@ -698,7 +698,7 @@ def run_dit_block(args, w):
 
 # Revision tag of the fine kernel; ncu traffic figures are only reported for
 # the revision they were captured on.
-KERNEL_REV = "fine-v6-static-producer-out"
+KERNEL_REV = "fine-v7-q-in-tmem-out"
 
 
 def main():

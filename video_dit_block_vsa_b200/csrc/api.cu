@@ -27,7 +27,7 @@ cudaError_t launch_coarse_only(const Geom&, int, float*, int32_t*, float*, const
                                cudaStream_t);
 cudaError_t launch_block_sparse_fwd(const Geom&, const FineMaps&, const int32_t*, const int32_t*,
                                     int, void*, float*, const float*, const float*, const float*,
-                                    bool, int*, int, cudaStream_t);
+                                    bool, int*, int, cudaStream_t, const void*);
 cudaError_t launch_debug_wait(uint64_t, int*, cudaStream_t);
 cudaError_t launch_linear_branch(int bh, long long N, int d, const void* q, const void* k,
                                  void* out, uint8_t* ws, const LinearLayout& L,
@@ -497,7 +497,7 @@ int vsa_block_sparse_fwd(const vsa_shape* shape, const void* q_tiled, const void
   if (fine_maps(g, q_tiled, k_tiled, v_tiled, &maps) != VSA_OK) return VSA_ERR_CUDA;
   return cuda_rc(launch_block_sparse_fwd(g, maps, cube_count, sel_idx, topk, o_fine_tiled,
                                          lse, nullptr, nullptr, nullptr, false, st.status, st.sms,
-                                         stream));
+                                         stream, q_tiled));
 }
 
 int vsa_block_sparse_fwd_out(const vsa_shape* shape, const void* q_tiled, const void* k_tiled,
@@ -527,7 +527,7 @@ int vsa_block_sparse_fwd_out(const vsa_shape* shape, const void* q_tiled, const 
   if (fine_maps(g, q_tiled, k_tiled, v_tiled, &maps) != VSA_OK) return VSA_ERR_CUDA;
   return cuda_rc(launch_block_sparse_fwd(g, maps, cube_count, sel_idx, topk, out, lse,
                                          g_fine ? o_coarse : nullptr, g_fine, g_coarse, true,
-                                         st.status, st.sms, stream));
+                                         st.status, st.sms, stream, q_tiled));
 }
 
 int vsa_select_transpose(const vsa_shape* shape, const int32_t* sel_idx, int topk,

@@ -23,16 +23,20 @@
 //  * Keys and values stream through a ring of 128-key smem slots (128-byte
 //    swizzle, TMA-filled) in exactly the order the MMA issuer consumes them:
 //    K_A0 K_B0 | V_A0 K_A1 V_B0 K_B1 | ...
-//  * TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+d),
-//    O_B [256+d, 256+2d).  The softmax writes P (bf16 pairs) over the first 64
-//    columns of its S, and O += P V reads P straight from TMEM (A operand in
-//    TMEM), so P never touches shared memory.  MMAs issued by one thread
-//    execute in order, so the next S = Q K^T cannot overwrite P before the
-//    P V that reads it.
-//  * M = 64 accumulators use TMEM lanes 0-15 of each warp's 32-lane
-//    sub-partition; the softmax reads them with the 16-lane .16x32bx2 shape:
-//    thread t holds row 16*(warp%4) + t%16, columns [64*(t/16), +64) of the
-//    step, i.e. exactly one key cube's 64 keys.
+//  * TMEM: an M = 64 accumulator occupies 16 lanes of each warp's 32-lane
+//    sub-partition, so the two cubes share columns: cube A in lanes 0-15,
+//    cube B in lanes 16-31.  Columns: S [0,128), O [128,128+d), Q
+//    [128+d, 128+3d/2).  The softmax warps write their cube's query rows into
+//    TMEM at the start of an item, and Q K^T reads Q as the TMEM A operand
+//    (no shared-memory operand reads for Q, and shared memory holds only the
+//    K/V ring: 7 slots at d = 128).  The softmax writes P (bf16 pairs) over
+//    the first 64 columns of its S, and O += P V reads P from TMEM as well, so
+//    P never touches shared memory.  MMAs issued by one thread execute in
+//    order, so the next S = Q K^T cannot overwrite P before the P V that
+//    reads it.
+//  * The softmax reads S with the 16-lane .16x32bx2 shape: thread t holds row
+//    16*(warp%4) + t%16, columns [64*(t/16), +64) of the step, i.e. exactly
+//    one key cube's 64 keys.
 //  * Online softmax in log2 units with conditional rescaling: the running
 //    reference max only moves (and O, l are rescaled) when a row's max grows
 //    by more than 2^8, so most steps skip the O round trip through registers.
@@ -70,12 +74,14 @@ struct Cfg {
   static constexpr uint32_t kQBytes = kHalves * kQHalf;        // one query cube tile
   static constexpr uint32_t kKVHalf = 128 * 128;               // [128 rows x 128 B]
   static constexpr uint32_t kSlotBytes = kHalves * kKVHalf;    // 128 keys x D
-  static constexpr int kSlots = D == 128 ? 5 : 10;
-  static constexpr uint32_t kRingOff = 4 * kQBytes;            // Q: 2 items x 2 cubes
+  static constexpr int kSlots = D == 128 ? 7 : 14;             // the ring fills shared memory
+  static constexpr uint32_t kRingOff = 0;
   static constexpr uint32_t kBarOff = kRingOff + kSlots * kSlotBytes;
-  static constexpr size_t kSmem = 1024 + kBarOff + 336;
-  static constexpr uint32_t kColS0 = 0, kColS1 = 128;
-  static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
+  static constexpr size_t kSmem = 1024 + kBarOff + 512;
+  // TMEM columns; cube A uses lanes 0-15 of every sub-partition, cube B lanes 16-31
+  static constexpr uint32_t kColS = 0;            // S (P over its first 64 columns)
+  static constexpr uint32_t kColO = 128;          // O
+  static constexpr uint32_t kColQ = 128 + D;      // Q, the A operand of Q K^T (D/2 columns)
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(64, D, false, true);  // P (TMEM), V MN-major
 };
 
@@ -95,6 +101,7 @@ struct Shared {
   volatile int* chunks;  // [2 Q buffers][2 cubes]: 16-row key chunks, producer -> MMA thread
   uint64_t* q_full;
   uint64_t* q_empty;
+  uint64_t* q_ready;  // [2] a cube's query rows are in TMEM
   uint64_t* kv_full;
   uint64_t* kv_empty;
   uint64_t* s_full;
@@ -103,6 +110,9 @@ struct Shared {
   volatile int* abort_flag;
   uint8_t* base;
 };
+
+// TMEM lane offset of cube c's accumulators and operands.
+__device__ __forceinline__ uint32_t cube_lanes(int c) { return static_cast<uint32_t>(16 * c) << 16; }
 
 struct Item {
   int bh, i0, i1, row0;
@@ -264,21 +274,13 @@ __device__ void producer(const Shared& sh, const Geom& g, const FineMaps& maps,
       n[c] = (T[c] + 7) / 8;
     }
     if (!it.has_b) T[1] = n[1] = 0;  // no cube B: nothing to plan or fetch
-    // ---- query tiles of both cubes
+    // ---- the item's chunk counts
     const int qb = t & 1;
     if (!wait_all(&sh.q_empty[qb], ((t >> 1) & 1) ^ 1)) return fail(sh, status);
     if (leader) {
       sh.chunks[2 * qb] = T[0];  // published to the MMA thread by the q_full arrive
       sh.chunks[2 * qb + 1] = it.has_b ? T[1] : 0;
-      mbar_arrive_expect_tx(&sh.q_full[qb], (it.has_b ? 2 : 1) * Cf::kQBytes);
-      uint8_t* qdst = sh.base + qb * 2 * Cf::kQBytes;
-#pragma unroll
-      for (int h = 0; h < Cf::kHalves; ++h) {
-        tma_load_2d(qdst + h * Cf::kQHalf, &maps.q, &sh.q_full[qb], h * 64, it.row0 + it.i0 * 64);
-        if (it.has_b)
-          tma_load_2d(qdst + Cf::kQBytes + h * Cf::kQHalf, &maps.q, &sh.q_full[qb], h * 64,
-                      it.row0 + it.i1 * 64);
-      }
+      mbar_arrive(&sh.q_full[qb]);  // the query rows go to TMEM through the softmax warps
     }
     // ---- key / value slots, in the MMA issuer's order: K_A0 K_B0, then per
     // step j: V_Aj K_A(j+1) V_Bj K_B(j+1), skipping steps a cube does not have.
@@ -378,7 +380,7 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
   uint32_t slot_c = 0, phase_c = 0;
   const uint64_t kdesc_base = sdesc_sw128(ring_base, 16, 1024);
   const uint64_t vdesc_base = sdesc_sw128(ring_base, Cf::kKVHalf, 1024);
-  uint32_t p_phase0 = 0u, p_phase1 = 0u;
+  uint32_t p_phase0 = 0u, p_phase1 = 0u, q_phase0 = 0u, q_phase1 = 0u;
   int t = 0;
   for (int item = blockIdx.x; item < items; item += gridDim.x, ++t) {
     if (*sh.abort_flag) return;
@@ -394,9 +396,6 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
       n[c] = (T + 7) / 8;
       last[c] = T - 8 * (n[c] - 1);
     }
-    const uint32_t qa0 = smem_u32(sh.base + qb * 2 * Cf::kQBytes);
-    const uint64_t qdesc0 = sdesc_sw128(qa0, 16, 1024);
-    const uint64_t qdesc1 = sdesc_sw128(qa0 + Cf::kQBytes, 16, 1024);
     auto next_slot = [&](uint32_t& slot) -> bool {
       slot = slot_c;
       if (!mbar_wait(&sh.kv_full[slot], phase_c)) return false;
@@ -407,20 +406,25 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
       tc_fence_after();
       return true;
     };
-    // S_c = Q_c K^T over one step's keys
+    // S_c = Q_c K^T over one step's keys; Q_c read from TMEM
     auto qk = [&](int c, int j) -> bool {
+      if (j == 0) {  // the cube's query rows are in TMEM
+        uint32_t& qp = c == 0 ? q_phase0 : q_phase1;
+        if (!mbar_wait(&sh.q_ready[c], qp)) return false;
+        qp ^= 1u;
+        tc_fence_after();
+      }
       uint32_t slot;
       if (!next_slot(slot)) return false;
-      const uint64_t a0 = c == 0 ? qdesc0 : qdesc1;
       const uint64_t b0 = kdesc_base + (slot * Cf::kSlotBytes >> 4);
       const int nc = j == (c ? n[1] : n[0]) - 1 ? (c ? last[1] : last[0]) : 8;
       const uint32_t idesc = (kIdescQK & ~(0x3Fu << 17)) | (static_cast<uint32_t>(2 * nc) << 17);
-      const uint32_t dS = tmem + (c == 0 ? Cf::kColS0 : Cf::kColS1);
+      const uint32_t dS = tmem + cube_lanes(c) + Cf::kColS;
+      const uint32_t aQ = tmem + cube_lanes(c) + Cf::kColQ;
 #pragma unroll
       for (int kk = 0; kk < kK; ++kk) {
-        const uint64_t ao = ((kk >> 2) * Cf::kQHalf + (kk & 3) * 32) >> 4;
         const uint64_t bo = ((kk >> 2) * Cf::kKVHalf + (kk & 3) * 32) >> 4;
-        umma_ss(dS, a0 + ao, b0 + bo, idesc, kk > 0 ? 1u : 0u);
+        umma_ts(dS, aQ + kk * 8, b0 + bo, idesc, kk > 0 ? 1u : 0u);
       }
       umma_commit(&sh.kv_empty[slot]);
       umma_commit(&sh.s_full[c]);
@@ -435,8 +439,8 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
       uint32_t slot;
       if (!next_slot(slot)) return false;
       const uint64_t v0 = vdesc_base + (slot * Cf::kSlotBytes >> 4);
-      const uint32_t dO = tmem + (c == 0 ? Cf::kColO0 : Cf::kColO1);
-      const uint32_t aP = tmem + (c == 0 ? Cf::kColS0 : Cf::kColS1);
+      const uint32_t dO = tmem + cube_lanes(c) + Cf::kColO;
+      const uint32_t aP = tmem + cube_lanes(c) + Cf::kColS;
       const int nsteps = c ? n[1] : n[0];
       const int nc = j == nsteps - 1 ? (c ? last[1] : last[0]) : 8;
       const uint32_t acc0 = j > 0 ? 1u : 0u;
@@ -476,7 +480,8 @@ __device__ void mma_issuer(const Shared& sh, const Geom& g, uint32_t tmem, int t
 template <int D, bool kTokenOut>
 __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c,
                            const int32_t* __restrict__ sel, int topk, const OutSpec os,
-                           int* status, const int32_t* __restrict__ counts) {
+                           int* status, const int32_t* __restrict__ counts,
+                           const __nv_bfloat16* __restrict__ q_tiled) {
   __nv_bfloat16* __restrict__ out = os.out;
   float* __restrict__ lse = os.lse;
   using Cf = Cfg<D>;
@@ -485,9 +490,10 @@ __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c
   const int wq = warp & 3;              // TMEM sub-partition of this warp
   const int hh = lane >> 4;             // which 64-key half of a step this thread holds
   const int r = wq * 16 + (lane & 15);  // query row of the cube
-  const uint32_t lane_addr = static_cast<uint32_t>(wq * 32) << 16;
-  const uint32_t tS = tmem + lane_addr + (c == 0 ? Cf::kColS0 : Cf::kColS1);
-  const uint32_t tO = tmem + lane_addr + (c == 0 ? Cf::kColO0 : Cf::kColO1);
+  const uint32_t lane_addr = (static_cast<uint32_t>(wq * 32) << 16) + cube_lanes(c);
+  const uint32_t tS = tmem + lane_addr + Cf::kColS;
+  const uint32_t tO = tmem + lane_addr + Cf::kColO;
+  const uint32_t tQ = tmem + lane_addr + Cf::kColQ;
   const float sl2 = kLog2e * rsqrtf(static_cast<float>(D));
   const int pairs = (g.C + 1) / 2;
   const int items = g.B * g.H * pairs;
@@ -500,6 +506,40 @@ __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c
     const int i = c == 0 ? it.i0 : it.i1;
     const int ni = cube_valid(g, i);
     const int32_t* list = sel + (static_cast<long long>(it.bh) * g.C + i) * topk;
+    {
+      // the cube's query rows into TMEM as the A operand of Q K^T (features
+      // 2 col, 2 col + 1 packed in column col): this thread's row r, features
+      // D/2 hh .. D/2 hh + D/2 - 1.  The previous item's products of this cube
+      // have completed: its last S and O were waited for.
+      const uint4* qrow = reinterpret_cast<const uint4*>(
+          q_tiled + (static_cast<long long>(it.row0) + i * 64 + r) * D + hh * (D / 2));
+      if constexpr (D == 128) {
+        uint32_t qw[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 x = __ldg(&qrow[u]);
+          qw[4 * u] = x.x;
+          qw[4 * u + 1] = x.y;
+          qw[4 * u + 2] = x.z;
+          qw[4 * u + 3] = x.w;
+        }
+        tmem_st_16x32bx2_x32(tQ, qw);
+      } else {
+        uint32_t qw[16];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint4 x = __ldg(&qrow[u]);
+          qw[4 * u] = x.x;
+          qw[4 * u + 1] = x.y;
+          qw[4 * u + 2] = x.z;
+          qw[4 * u + 3] = x.w;
+        }
+        tmem_st_16x32bx2_x16(tQ, qw);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sh.q_ready[c]);
+    }
     float m_ref = -INFINITY, l_part = 0.f;
     const int W = count_wide(g, list, topk, lane, nullptr);
     const int T = 3 * W + topk;  // 16-row key chunks of the cube
@@ -664,7 +704,8 @@ __device__ void softmax_wg(const Shared& sh, const Geom& g, uint32_t tmem, int c
 template <int D, bool kTokenOut>
 __global__ void __launch_bounds__(kThreads, 1) fine_fwd_kernel(
     const __grid_constant__ FineMaps maps, Geom g, const int32_t* __restrict__ counts,
-    const int32_t* __restrict__ sel, int topk, const OutSpec os, int* status) {
+    const int32_t* __restrict__ sel, int topk, const OutSpec os, int* status,
+    const __nv_bfloat16* __restrict__ q_tiled) {
   using Cf = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -679,7 +720,8 @@ __global__ void __launch_bounds__(kThreads, 1) fine_fwd_kernel(
   sh.s_full = bars + 4 + 2 * Cf::kSlots;
   sh.p_full = sh.s_full + 2;
   sh.o_full = sh.s_full + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sh.o_full + 2);
+  sh.q_ready = sh.s_full + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sh.q_ready + 2);
   sh.abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   sh.chunks = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
@@ -695,6 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_fwd_kernel(
       mbar_init(&sh.s_full[q], 1);
       mbar_init(&sh.p_full[q], 128);
       mbar_init(&sh.o_full[q], 1);
+      mbar_init(&sh.q_ready[q], 128);
     }
     for (int s = 0; s < Cf::kSlots; ++s) {
       mbar_init(&sh.kv_full[s], 1);
@@ -718,7 +761,8 @@ __global__ void __launch_bounds__(kThreads, 1) fine_fwd_kernel(
   } else if (warp == kMmaWarp) {
     if (lane == 0) mma_issuer<D>(sh, g, tmem, topk, status);
   } else if (warp >= kSoftmaxWarp0) {
-    softmax_wg<D, kTokenOut>(sh, g, tmem, (warp - kSoftmaxWarp0) >> 2, sel, topk, os, status, counts);
+    softmax_wg<D, kTokenOut>(sh, g, tmem, (warp - kSoftmaxWarp0) >> 2, sel, topk, os, status, counts,
+                             q_tiled);
   }
   tc_fence_before();
   __syncthreads();
@@ -733,7 +777,7 @@ cudaError_t launch_block_sparse_fwd(const Geom& g, const FineMaps& maps, const i
                                     const int32_t* sel, int topk, void* out, float* lse,
                                     const float* o_coarse, const float* g_fine,
                                     const float* g_coarse, bool token_order, int* status, int sms,
-                                    cudaStream_t s) {
+                                    cudaStream_t s, const void* q_tiled) {
   const long long items = static_cast<long long>(g.B) * g.H * ((g.C + 1) / 2);
   const int grid = static_cast<int>(items < sms ? items : sms);
   const size_t smem = fine_smem_bytes(g.d);
@@ -745,7 +789,8 @@ cudaError_t launch_block_sparse_fwd(const Geom& g, const FineMaps& maps, const i
   auto run = [&](auto kernel, int which) -> cudaError_t {
     cudaError_t e = smem_limit_once(kernel, static_cast<int>(smem), &limit_set[which]);
     if (e != cudaSuccess) return e;
-    kernel<<<grid, kThreads, smem, s>>>(maps, g, counts, sel, topk, os, status);
+    kernel<<<grid, kThreads, smem, s>>>(maps, g, counts, sel, topk, os, status,
+                                        static_cast<const __nv_bfloat16*>(q_tiled));
     return cudaSuccess;
   };
   if (g.d == 128)
