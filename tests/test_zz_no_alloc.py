@@ -85,3 +85,70 @@ def test_noalloc_rejects_problems_beyond_its_scratch(vsa):
     assert rc == vsa.VSA_ERR_TOO_LARGE
     assert "scratch" in vsa.vsa_strerror(rc)
     assert vsa.vsa_get_status() == 0
+
+
+def test_noalloc_under_a_second_context(vsa):
+    """The entry point called while a second CUDA context, made with the driver
+    API as a host application might, is current: the library looks up its
+    scratch array and status word for that context, so the result equals the
+    primary context's bit for bit, and the primary context still works after
+    the second one is gone."""
+    from cuda.bindings import driver as drv
+
+    w = wl.WORKLOADS["tiny_k2"]
+    shape, bufs = _tiled_inputs(vsa, w)
+    C = vsa.vsa_num_cubes(shape)
+    B, H, d, k = w.batch, w.heads, w.head_dim, w.topk
+    sel_ref = torch.empty(B, H, C, k, dtype=torch.int32, device="cuda")
+    oc_ref = torch.empty(B, H, C, d, dtype=torch.float32, device="cuda")
+    lg_ref = torch.empty(B, H, C, C, dtype=torch.float32, device="cuda")
+    assert _noalloc_call(vsa, shape, bufs, k, sel_ref, oc_ref, lg_ref) == 0
+    torch.cuda.synchronize()
+    host = [t.cpu().numpy() for t in (bufs.q_t.view(torch.int16), bufs.k_t.view(torch.int16),
+                                      bufs.v_t.view(torch.int16), bufs.counts)]
+    ok = drv.CUresult.CUDA_SUCCESS
+    err, dev = drv.cuDeviceGet(torch.cuda.current_device())
+    assert err == ok
+    err, ctx = drv.cuCtxCreate(0, dev)
+    assert err == ok
+    try:
+        ptrs = []
+
+        def alloc(nbytes):
+            e, p = drv.cuMemAlloc(nbytes)
+            assert e == ok
+            ptrs.append(p)
+            return p
+
+        dins = []
+        for a in host:
+            p = alloc(a.nbytes)
+            assert drv.cuMemcpyHtoD(p, a, a.nbytes)[0] == ok
+            dins.append(p)
+        sel = np.empty((B, H, C, k), np.int32)
+        oc = np.empty((B, H, C, d), np.float32)
+        lg = np.empty((B, H, C, C), np.float32)
+        sel_p, oc_p, lg_p = alloc(sel.nbytes), alloc(oc.nbytes), alloc(lg.nbytes)
+        vp = lambda p: ctypes.c_void_p(int(p))
+        rc = vsa._lib.vsa_coarse_select_noalloc(ctypes.byref(shape), vp(dins[0]), vp(dins[1]),
+                                                vp(dins[2]), vp(dins[3]), k, vp(oc_p), vp(sel_p),
+                                                vp(lg_p), None)
+        assert rc == 0
+        assert drv.cuCtxSynchronize()[0] == ok
+        assert vsa._lib.vsa_get_status(None) == 0
+        for a, p in ((sel, sel_p), (oc, oc_p), (lg, lg_p)):
+            assert drv.cuMemcpyDtoH(a, p, a.nbytes)[0] == ok
+        for p in ptrs:
+            assert drv.cuMemFree(p)[0] == ok
+    finally:
+        drv.cuCtxPopCurrent()
+        drv.cuCtxDestroy(ctx)
+    assert np.array_equal(sel, sel_ref.cpu().numpy())
+    assert np.array_equal(oc, oc_ref.cpu().numpy())
+    assert np.array_equal(lg, lg_ref.cpu().numpy())
+    # back in the primary context
+    sel2 = torch.empty_like(sel_ref)
+    assert _noalloc_call(vsa, shape, bufs, k, sel2, torch.empty_like(oc_ref), torch.empty_like(lg_ref)) == 0
+    torch.cuda.synchronize()
+    assert vsa.vsa_get_status() == 0
+    assert torch.equal(sel2, sel_ref)

@@ -45,7 +45,8 @@ cudaError_t launch_coarse_backward(int, int, int, const float*, const float*, co
 size_t coarse_backward_plane_bytes(int C);
 cudaError_t launch_block_sparse_bwd(const Geom&, const BwdMaps&, int, const float*, const float*,
                                     const int32_t*, const int32_t*, const int32_t*, const float*,
-                                    void*, void*, void*, int*, int, cudaStream_t);
+                                    void*, void*, void*, int*, int, cudaStream_t, const void*,
+                                    const void*);
 
 // Device-side status word, one per device that loads the library.
 __device__ int g_status;
@@ -627,7 +628,7 @@ int vsa_block_sparse_bwd(const vsa_shape* shape, const void* q_tiled, const void
     return VSA_ERR_CUDA;
   return cuda_rc(launch_block_sparse_bwd(g, maps, topk, lse, delta, sel_idx, key_offsets,
                                          query_lists, d_pooled, dq, dk, dv, st.status, st.sms,
-                                         stream));
+                                         stream, q_tiled, do_fine_tiled));
 }
 
 int vsa_get_status(cudaStream_t stream) {

@@ -70,6 +70,8 @@ struct BCfg {
   // TMEM: S, dP of buffer b at columns 128 b and 128 b + 64; accumulators after
   static constexpr uint32_t kAcc0 = 256;                   // dQ (dq) or dK (dkdv)
   static constexpr uint32_t kAcc1 = 256 + D;               // dV (dkdv)
+  static constexpr uint32_t kColQ = 256 + D;               // dq: Q_i, the A operand of S
+  static constexpr uint32_t kColG = 256 + D + D / 2;       // dq: dO_i, the A operand of dP
   static constexpr uint32_t kIdescS = idesc_bf16_f32(64, 64, false, false);
   static constexpr uint32_t kIdescAcc = idesc_bf16_f32(64, D, false, true);
 };
@@ -102,6 +104,8 @@ struct BwdArgs {
   const float* bar1;           // dkdv: dvbar
   bf16* out0;                  // dq: dq; dkdv: dk  (token order)
   bf16* out1;                  // dkdv: dv
+  const bf16* qt;              // dq: tiled q (rows copied into TMEM)
+  const bf16* dot;             // dq: tiled dO_f
   int* status;
 };
 
@@ -193,18 +197,20 @@ __device__ void bwd_producer(const BwdShared& sh, const BwdArgs& a, const BwdMap
     const int n = item_list<kDq>(a, bh, cube, &list);
     if (n == 0) continue;
     const int row0 = bh * static_cast<int>(g.rows);
-    const int sb = u & 1;
-    if (!wait_all(&sh.stat_empty[sb], ((u >> 1) & 1) ^ 1)) return bwd_fail(sh, a.status);
-    ++u;
-    // the stationary pair: Q_i, dO_i (dq) or K_j, V_j (dkdv)
-    uint8_t* stat = sh.base + sb * Cf::kStat;
-    if (lane == 0) mbar_arrive_expect_tx(&sh.stat_full[sb], Cf::kStat);
-    __syncwarp();
-    if (lane < 2 * Cf::kHalves) {
-      const int which = lane / Cf::kHalves, h = lane - which * Cf::kHalves;
-      const CUtensorMap* m = kDq ? (which ? &maps.dO : &maps.q) : (which ? &maps.v : &maps.k);
-      tma_load_2d(stat + which * Cf::kTile + h * Cf::kHalf, m, &sh.stat_full[sb], h * 64,
-                  row0 + cube * 64);
+    if (!kDq) {
+      // the stationary pair K_j, V_j (the dq kernel's Q_i, dO_i go to TMEM
+      // through the elementwise warps)
+      const int sb = u & 1;
+      if (!wait_all(&sh.stat_empty[sb], ((u >> 1) & 1) ^ 1)) return bwd_fail(sh, a.status);
+      ++u;
+      uint8_t* stat = sh.base + sb * Cf::kStat;
+      if (lane == 0) mbar_arrive_expect_tx(&sh.stat_full[sb], Cf::kStat);
+      __syncwarp();
+      if (lane < 2 * Cf::kHalves) {
+        const int which = lane / Cf::kHalves, h = lane - which * Cf::kHalves;
+        tma_load_2d(stat + which * Cf::kTile + h * Cf::kHalf, which ? &maps.v : &maps.k,
+                    &sh.stat_full[sb], h * 64, row0 + cube * 64);
+      }
     }
     // the streamed pair of every step: K_j, V_j (dq) or Q_i, dO_i and the
     // lse and delta rows of query cube i (dkdv)
@@ -272,12 +278,18 @@ __device__ void bwd_mma(const BwdShared& sh, const BwdArgs& a, uint32_t tmem) {
 #pragma unroll
       for (int kk = 0; kk < kK; ++kk) {
         const uint64_t o = ((kk >> 2) * Cf::kHalf + (kk & 3) * 32) >> 4;
-        umma_ss(tmem + col_s(b), a0 + o, b0 + o, Cf::kIdescS, kk > 0 ? 1u : 0u);
+        if (kDq)  // Q_i from TMEM: 16 features = 8 packed columns per k-step
+          umma_ts(tmem + col_s(b), tmem + Cf::kColQ + kk * 8, b0 + o, Cf::kIdescS, kk > 0 ? 1u : 0u);
+        else
+          umma_ss(tmem + col_s(b), a0 + o, b0 + o, Cf::kIdescS, kk > 0 ? 1u : 0u);
       }
 #pragma unroll
       for (int kk = 0; kk < kK; ++kk) {
         const uint64_t o = ((kk >> 2) * Cf::kHalf + (kk & 3) * 32) >> 4;
-        umma_ss(tmem + col_p(b), a1 + o, b1 + o, Cf::kIdescS, kk > 0 ? 1u : 0u);
+        if (kDq)
+          umma_ts(tmem + col_p(b), tmem + Cf::kColG + kk * 8, b1 + o, Cf::kIdescS, kk > 0 ? 1u : 0u);
+        else
+          umma_ss(tmem + col_p(b), a1 + o, b1 + o, Cf::kIdescS, kk > 0 ? 1u : 0u);
       }
       umma_commit(&sh.s_full[b]);
       return true;
@@ -390,6 +402,44 @@ __device__ void bwd_elementwise(const BwdShared& sh, const BwdArgs& a, uint32_t 
         const long long row = static_cast<long long>(bh) * g.rows + cube * 64 + r;
         lse2 = __ldg(&a.lse[row]) * kLog2e;
         dlt = __ldg(&a.delta[row]);
+      }
+      if (kDq) {
+        // Q_i and dO_i rows into TMEM as the A operands of S and dP: this
+        // thread's row r, features D/2 h .. D/2 h + D/2 - 1 (two per column).
+        // The previous item's products have completed: its accumulator was
+        // waited for.
+        const long long row = static_cast<long long>(bh) * g.rows + cube * 64 + r;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          const uint4* src = reinterpret_cast<const uint4*>((which ? a.dot : a.qt) + row * D + h * (D / 2));
+          const uint32_t col = which ? Cf::kColG : Cf::kColQ;
+          if constexpr (D == 128) {
+            uint32_t w[32];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+              const uint4 v4 = __ldg(&src[x]);
+              w[4 * x] = v4.x;
+              w[4 * x + 1] = v4.y;
+              w[4 * x + 2] = v4.z;
+              w[4 * x + 3] = v4.w;
+            }
+            tmem_st_16x32bx2_x32(tmem + lane_addr + col, w);
+          } else {
+            uint32_t w[16];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              const uint4 v4 = __ldg(&src[x]);
+              w[4 * x] = v4.x;
+              w[4 * x + 1] = v4.y;
+              w[4 * x + 2] = v4.z;
+              w[4 * x + 3] = v4.w;
+            }
+            tmem_st_16x32bx2_x16(tmem + lane_addr + col, w);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sh.stat_full[u & 1]);
       }
       ListWindow win;
       win.init(list, n, lane);
@@ -511,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1) fine_bwd_kernel(const __grid_cons
   }
   if (threadIdx.x == 0) {
     for (int q = 0; q < 2; ++q) {
-      mbar_init(&sh.stat_full[q], 1);
+      mbar_init(&sh.stat_full[q], kDq ? kEwThreads : 1);
       mbar_init(&sh.stat_empty[q], 1);
       mbar_init(&sh.s_full[q], 1);
       mbar_init(&sh.ds_full[q], kEwThreads);
@@ -580,8 +630,11 @@ cudaError_t launch_block_sparse_bwd(const Geom& g, const BwdMaps& maps, int topk
                                     const float* lse, const float* delta, const int32_t* sel,
                                     const int32_t* key_offsets, const int32_t* query_lists,
                                     const float* dpooled, void* dq, void* dk, void* dv,
-                                    int* status, int sms, cudaStream_t s) {
+                                    int* status, int sms, cudaStream_t s, const void* q_tiled,
+                                    const void* do_tiled) {
   BwdArgs a{};
+  a.qt = static_cast<const bf16*>(q_tiled);
+  a.dot = static_cast<const bf16*>(do_tiled);
   a.g = g;
   a.topk = topk;
   a.sel = sel;
