@@ -19,7 +19,7 @@ from video_dit_block_vsa_b200 import vsa as V  # noqa: E402
 
 HOST_ONLY = {"vsa_num_cubes", "vsa_topk_from_ratio", "vsa_workspace_bytes",
              "vsa_forward_host_workspace_bytes", "vsa_coarse_backward_workspace_bytes",
-             "vsa_strerror"}
+             "vsa_linear_workspace_bytes", "vsa_strerror"}
 
 
 class Recorder:
@@ -149,3 +149,46 @@ def test_device_buffers_are_checked():
         V._expect(torch.zeros(4, dtype=torch.int32), torch.int32, (4,), "cube_count")
     with pytest.raises(ValueError, match="contiguous"):
         V._ptr(torch.zeros(4, 4).t())
+
+
+@pytest.mark.parametrize("gated", [True, False])
+def test_attention_block_wiring(lib, gated):
+    """QKV projection into the tiled buffers, coarse stage and fine stage on
+    them, the combine when gated, and the output projection reading the tiled
+    attention output (the combined one when gated)."""
+    shape, topk, (_, _, _, _, _, g_f, g_c), bufs = setup(gated)
+    hidden = 128
+    x = torch.zeros(1, 256, hidden, dtype=torch.bfloat16)
+    w_qkv = torch.zeros(3 * 2 * 64, hidden, dtype=torch.bfloat16)
+    w_o = torch.zeros(hidden, 2 * 64, dtype=torch.bfloat16)
+    y = torch.zeros(1, 256, hidden, dtype=torch.bfloat16)
+    V.vsa_attention_block(shape, hidden, x, w_qkv, w_o, topk, y, g_f, g_c, bufs=bufs)
+    expect = ["vsa_qkv_projection_tiled", "vsa_coarse_select", "vsa_block_sparse_fwd"] + \
+             (["vsa_combine"] if gated else []) + ["vsa_out_projection_tiled"]
+    assert lib.names() == expect
+    calls = dict(lib.calls)
+    qkv = calls["vsa_qkv_projection_tiled"]  # (shape, hidden, x, w, q_t, k_t, v_t, counts, stream)
+    assert qkv[1] == hidden
+    assert [addr(a) for a in qkv[4:8]] == [ptr(bufs.q_t), ptr(bufs.k_t), ptr(bufs.v_t), ptr(bufs.counts)]
+    outp = calls["vsa_out_projection_tiled"]  # (shape, hidden, o_t, w_o, y, stream)
+    assert addr(outp[2]) == ptr(bufs.out_t if gated else bufs.o_f)
+    assert addr(outp[4]) == ptr(y)
+
+
+def test_linear_branch_marshalling(lib):
+    shape, _, (q, k, v, out, _, _, _), _ = setup(False)
+    ws = torch.zeros(V.vsa_linear_workspace_bytes(shape), dtype=torch.uint8)
+    V.vsa_linear_branch_add(shape, q, k, v, out, ws)
+    (name, args), = lib.calls
+    assert name == "vsa_linear_branch_add"
+    assert [addr(a) for a in args[1:6]] == [ptr(q), ptr(k), ptr(v), ptr(out), ptr(ws)]
+    assert args[6] == ws.numel()
+
+
+def test_head_parallel_one_rank_runs_the_fused_forward(lib):
+    from video_dit_block_vsa_b200 import head_parallel as hp
+    _, topk, (q, k, v, _, _, g_f, g_c), _ = setup(True)
+    hp.vsa_forward_head_parallel((4, 8, 8), topk, q, k, v, g_f, g_c)
+    assert lib.names() == ["vsa_tile_permute_pool", "vsa_coarse_select_pooled",
+                           "vsa_block_sparse_fwd_out"]
+
